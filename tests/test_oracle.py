@@ -1,0 +1,400 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+* the KV-cache sizes printed on the pages (``tests/golden/kv_cache_sizes.txt``);
+* closed forms (two-key sigmoid example, identical keys, causal row 0, one key, q = 0);
+* scalar brute force on tiny inputs (the 2x2x3 toy and small random shapes);
+* the MHA (Hkv = Hq) and MQA (Hkv = 1) reductions, per head, by brute force;
+* the tiled online-softmax of CSDN «注意力变体深挖» §6.2 at several block sizes;
+* torch's float64 CPU ``scaled_dot_product_attention(enable_gqa=True)``;
+* invariants (key shift, value affine map, key permutation, LSE bounds, decode = last
+  causal row, paged = contiguous);
+* planted mistakes (wrong head mapping, dropped scale, top-left causal alignment) that
+  the pins above must catch.
+"""
+
+import math
+import os
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import oracle.attention as oatt
+from oracle import (
+    attention_ref,
+    attention_rows_ref,
+    brute_force_attention,
+    decode_ref,
+    flash_blockwise_ref,
+    kv_cache_bytes_ref,
+    paged_pool_blocks_ref,
+    decode_plan_ref,
+)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed):
+    return np.random.Generator(np.random.PCG64(seed)).standard_normal(shape)
+
+
+def _bf(a):
+    return brute_force_attention(a[0].tolist(), a[1].tolist(), a[2].tolist(), **a[3])
+
+
+# ---------------------------------------------------------------- KV cache sizing
+
+
+def _golden_rows():
+    rows = []
+    with open(os.path.join(GOLDEN, "kv_cache_sizes.txt"), encoding="utf-8") as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            nums, src = line.split("|", 1)
+            vals = [int(x) for x in nums.split()]
+            rows.append((vals, src.strip()))
+    return rows
+
+
+@pytest.mark.parametrize("row", _golden_rows(), ids=lambda r: r[1][:40])
+def test_kv_cache_sizes_from_pages(row):
+    (layers, hkv, d, seq, batch, eb, expected), _src = row
+    assert kv_cache_bytes_ref(layers, hkv, d, seq, batch, eb) == expected
+
+
+def test_kv_cache_batch_factor():
+    # kongchang course summary: the cache grows linearly with the batch b.
+    assert kv_cache_bytes_ref(32, 8, 128, 4096, 3, 2) == 3 * 536870912
+
+
+def test_paged_pool_blocks_hand_example():
+    # ceil(0/16)+ceil(1/16)+ceil(16/16)+ceil(17/16)+ceil(33/16) = 0+1+1+2+3
+    assert paged_pool_blocks_ref([0, 1, 16, 17, 33], 16) == 7
+    assert paged_pool_blocks_ref([5], 1) == 5
+
+
+# ---------------------------------------------------------------- closed forms
+
+
+def test_two_key_sigmoid_example():
+    # scores (scale s): s*2 and 0 -> weights sigmoid(2s), 1 - sigmoid(2s).
+    q = np.array([1.0, 0.0, 0.0]).reshape(1, 1, 1, 3)
+    k = np.array([[2.0, 0.0, 0.0], [0.0, 0.0, 0.0]]).reshape(1, 1, 2, 3)
+    v = np.array([[1.0, 0.0, 0.0], [0.0, 1.0, 0.0]]).reshape(1, 1, 2, 3)
+    for s in (1.0, 0.5):
+        o, lse = attention_ref(q, k, v, scale=s)
+        w0 = 1.0 / (1.0 + math.exp(-2.0 * s))
+        np.testing.assert_allclose(o[0, 0, 0], [w0, 1.0 - w0, 0.0], rtol=0, atol=1e-15)
+        assert abs(lse[0, 0, 0] - math.log(math.exp(2.0 * s) + 1.0)) < 1e-14
+    o, lse = attention_ref(q, k, v)  # default scale 1/sqrt(3)
+    w0 = 1.0 / (1.0 + math.exp(-2.0 / math.sqrt(3.0)))
+    assert abs(o[0, 0, 0, 0] - w0) < 1e-15
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_identical_keys_give_uniform_weights(causal):
+    B, Hq, Hkv, S, D = 2, 4, 2, 9, 6
+    q = _rand((B, Hq, S, D), 1)
+    u = _rand((D,), 2)
+    k = np.broadcast_to(u, (B, Hkv, S, D)).copy()
+    v = _rand((B, Hkv, S, D), 3)
+    o, lse = attention_ref(q, k, v, causal=causal, scale=0.3)
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(S):
+                n = i + 1 if causal else S
+                np.testing.assert_allclose(o[b, h, i], v[b, h // 2, :n].mean(axis=0), atol=1e-13)
+                s = 0.3 * float(q[b, h, i] @ u)
+                assert abs(lse[b, h, i] - (s + math.log(n))) < 1e-12
+
+
+def test_causal_row0_is_v0():
+    B, Hq, Hkv, S, D = 1, 4, 2, 11, 5
+    q, k, v = _rand((B, Hq, S, D), 4), _rand((B, Hkv, S, D), 5), _rand((B, Hkv, S, D), 6)
+    o, lse = attention_ref(q, k, v, causal=True, scale=0.7)
+    for h in range(Hq):
+        np.testing.assert_allclose(o[0, h, 0], v[0, h // 2, 0], atol=1e-15)
+        assert abs(lse[0, h, 0] - 0.7 * float(q[0, h, 0] @ k[0, h // 2, 0])) < 1e-13
+
+
+def test_single_key_returns_v0():
+    q, k, v = _rand((2, 2, 3, 4), 7), _rand((2, 1, 1, 4), 8), _rand((2, 1, 1, 4), 9)
+    o, lse = attention_ref(q, k, v, scale=0.5)
+    for b in range(2):
+        for h in range(2):
+            np.testing.assert_allclose(o[b, h], np.broadcast_to(v[b, 0, 0], (3, 4)), atol=1e-15)
+            np.testing.assert_allclose(lse[b, h], 0.5 * (q[b, h] @ k[b, 0, 0]), atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_is_mean_of_values(causal):
+    S = 7
+    q = np.zeros((1, 2, S, 3))
+    k, v = _rand((1, 1, S, 3), 10), _rand((1, 1, S, 3), 11)
+    o, lse = attention_ref(q, k, v, causal=causal)
+    for i in range(S):
+        n = i + 1 if causal else S
+        np.testing.assert_allclose(o[0, 1, i], v[0, 0, :n].mean(axis=0), atol=1e-15)
+        assert abs(lse[0, 0, i] - math.log(n)) < 1e-15
+
+
+def test_large_scores_stay_finite():
+    # max-subtracted softmax (CSDN §五): scores near 1e3 must not overflow.
+    q = np.full((1, 1, 2, 2), 30.0)
+    k = np.array([[[[30.0, 30.0], [29.0, 29.0]]]])
+    v = np.array([[[[1.0, 0.0], [0.0, 1.0]]]])
+    o, lse = attention_ref(q, k, v, scale=1.0)  # scores 1800 and 1740
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    np.testing.assert_allclose(o[0, 0, 0], [1.0, math.exp(-60.0)], rtol=1e-12)
+
+
+# ---------------------------------------------------------------- brute force
+
+
+@pytest.mark.parametrize("hkv", [1, 2])
+@pytest.mark.parametrize("causal", [False, True])
+def test_toy_2x2x3_brute_force(hkv, causal):
+    q, k, v = _rand((1, 2, 2, 3), 12), _rand((1, hkv, 2, 3), 13), _rand((1, hkv, 2, 3), 14)
+    o, lse = attention_ref(q, k, v, causal=causal)
+    ob, lb = _bf((q, k, v, dict(causal=causal)))
+    np.testing.assert_allclose(o, np.array(ob), atol=1e-14, rtol=0)
+    np.testing.assert_allclose(lse, np.array(lb), atol=1e-14, rtol=0)
+
+
+SMALL = [
+    # B, Hq, Hkv, Sq, Sk, D, causal
+    (1, 4, 2, 5, 5, 3, False),
+    (2, 4, 2, 5, 5, 3, True),
+    (1, 6, 3, 3, 7, 4, True),   # Sq < Sk: bottom-right causal alignment
+    (1, 4, 1, 6, 4, 2, True),   # Sq > Sk: first rows fully masked
+    (1, 3, 3, 4, 6, 5, False),  # MHA
+    (2, 8, 1, 2, 3, 4, False),  # MQA
+]
+
+
+@pytest.mark.parametrize("shape", SMALL)
+def test_random_small_vs_brute_force(shape):
+    B, Hq, Hkv, Sq, Sk, D, causal = shape
+    seed = sum(shape[:6])
+    q, k, v = _rand((B, Hq, Sq, D), seed), _rand((B, Hkv, Sk, D), seed + 1), _rand((B, Hkv, Sk, D), seed + 2)
+    o, lse = attention_ref(q, k, v, causal=causal, scale=0.6)
+    ob, lb = _bf((q, k, v, dict(causal=causal, scale=0.6)))
+    np.testing.assert_allclose(o, np.array(ob), atol=1e-13, rtol=0)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(np.array(lb)))
+    fin = np.isfinite(lse)
+    np.testing.assert_allclose(lse[fin], np.array(lb)[fin], atol=1e-13, rtol=0)
+
+
+def test_fully_masked_rows_are_zero_with_neg_inf_lse():
+    q, k, v = _rand((1, 2, 6, 3), 20), _rand((1, 1, 4, 3), 21), _rand((1, 1, 4, 3), 22)
+    o, lse = attention_ref(q, k, v, causal=True)
+    # key j allowed for row i iff j <= i + 4 - 6: rows 0 and 1 see nothing.
+    assert np.all(o[0, :, :2] == 0.0) and np.all(np.isneginf(lse[0, :, :2]))
+    assert np.all(np.isfinite(lse[0, :, 2:]))
+    np.testing.assert_allclose(o[0, :, 2], np.broadcast_to(v[0, 0, 0], (2, 3)), atol=1e-15)
+
+
+def test_mha_reduction_per_head():
+    # gocoding §3 / CSDN §四: G = H reduces GQA to MHA (each head its own K/V).
+    H, S, D = 3, 4, 3
+    q, k, v = _rand((1, H, S, D), 30), _rand((1, H, S, D), 31), _rand((1, H, S, D), 32)
+    o, _ = attention_ref(q, k, v, causal=True)
+    for h in range(H):
+        ob, _ = brute_force_attention(q[:, h : h + 1].tolist(), k[:, h : h + 1].tolist(),
+                                      v[:, h : h + 1].tolist(), causal=True)
+        np.testing.assert_allclose(o[:, h : h + 1], np.array(ob), atol=1e-14)
+
+
+def test_mqa_reduction_per_head():
+    # gocoding §2 / CSDN §三: G = 1 -- every query head uses the single K/V head.
+    H, S, D = 4, 5, 2
+    q, k, v = _rand((1, H, S, D), 33), _rand((1, 1, S, D), 34), _rand((1, 1, S, D), 35)
+    o, _ = attention_ref(q, k, v)
+    for h in range(H):
+        ob, _ = brute_force_attention(q[:, h : h + 1].tolist(), k.tolist(), v.tolist())
+        np.testing.assert_allclose(o[:, h : h + 1], np.array(ob), atol=1e-14)
+
+
+# ---------------------------------------------------------------- tiled online softmax (§6.2)
+
+
+@pytest.mark.parametrize("bq,bkv", [(1, 1), (7, 7), (32, 32), (64, 64), (5, 32), (64, 13)])
+def test_blockwise_online_softmax_equals_one_shot(bq, bkv):
+    nq, nk, d = 64, 80, 16
+    q, k, v = _rand((nq, d), 40) * 2, _rand((nk, d), 41) * 2, _rand((nk, d), 42)
+    ob, lb = flash_blockwise_ref(q, k, v, bq, bkv, scale=0.5)
+    o, lse = attention_ref(q[None, None], k[None, None], v[None, None], scale=0.5)
+    np.testing.assert_allclose(ob, o[0, 0], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lb, lse[0, 0], atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------- torch fp64 cross-check
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_torch_sdpa_float64_crosscheck(causal):
+    # The tiny exact-attention case: B=1, Hq=4, Hkv=2, S=128, D=64, seed 0.
+    from exact_attention_137_b200.workloads import prefill_inputs, to_f64
+
+    x = prefill_inputs(1, 4, 2, 128, 128, 64, dtype="f32", seed=0)
+    q, k, v = (to_f64(x[n]) for n in ("q", "k", "v"))
+    o, lse = attention_ref(q, k, v, causal=causal, scale=1 / 8)
+    ot = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v),
+        is_causal=causal, scale=1 / 8, enable_gqa=True)
+    np.testing.assert_allclose(o, ot.numpy(), atol=1e-12, rtol=0)
+    # LSE by an independent route: log of torch's float64 logsumexp of the masked scores.
+    kr = torch.from_numpy(k).repeat_interleave(2, dim=1)
+    s = torch.from_numpy(q) @ kr.transpose(-1, -2) / 8
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(128, 128, dtype=torch.bool), 1), float("-inf"))
+    np.testing.assert_allclose(lse, torch.logsumexp(s, -1).numpy(), atol=1e-12, rtol=0)
+
+
+# ---------------------------------------------------------------- invariants
+
+
+def test_key_shift_invariance():
+    q, k, v = _rand((1, 4, 8, 5), 50), _rand((1, 2, 8, 5), 51), _rand((1, 2, 8, 5), 52)
+    u = _rand((5,), 53)
+    o1, l1 = attention_ref(q, k, v, causal=True, scale=0.4)
+    o2, l2 = attention_ref(q, k + u, v, causal=True, scale=0.4)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+    np.testing.assert_allclose(l2 - l1, 0.4 * np.einsum("bhsd,d->bhs", q, u), atol=1e-12)
+
+
+def test_value_affine_map():
+    q, k, v = _rand((1, 2, 6, 4), 54), _rand((1, 1, 6, 4), 55), _rand((1, 1, 6, 4), 56)
+    o1, _ = attention_ref(q, k, v, causal=True)
+    o2, _ = attention_ref(q, k, 3.0 * v - 2.0, causal=True)
+    np.testing.assert_allclose(o2, 3.0 * o1 - 2.0, atol=1e-12)
+
+
+def test_key_permutation_invariance_noncausal():
+    q, k, v = _rand((1, 2, 5, 3), 57), _rand((1, 2, 9, 3), 58), _rand((1, 2, 9, 3), 59)
+    perm = np.random.Generator(np.random.PCG64(60)).permutation(9)
+    o1, l1 = attention_ref(q, k, v)
+    o2, l2 = attention_ref(q, k[:, :, perm], v[:, :, perm])
+    np.testing.assert_allclose(o1, o2, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, atol=1e-13)
+
+
+def test_lse_bounds():
+    q, k, v = _rand((1, 2, 16, 4), 61) * 3, _rand((1, 2, 16, 4), 62), _rand((1, 2, 16, 4), 63)
+    _, lse = attention_ref(q, k, v, causal=True, scale=1.0)
+    s = np.einsum("bhid,bhjd->bhij", q, k)
+    for i in range(16):
+        mx = s[0, :, i, : i + 1].max(axis=1)
+        assert np.all(lse[0, :, i] >= mx - 1e-12)
+        assert np.all(lse[0, :, i] <= mx + math.log(i + 1) + 1e-12)
+
+
+def test_rows_subset_equals_full_rows():
+    q, k, v = _rand((2, 4, 12, 3), 64), _rand((2, 2, 12, 3), 65), _rand((2, 2, 12, 3), 66)
+    rows = np.array([0, 3, 11, 7])
+    o, lse = attention_ref(q, k, v, causal=True)
+    os_, ls = attention_rows_ref(q, k, v, causal=True, rows=rows)
+    np.testing.assert_array_equal(os_, o[:, :, rows])
+    np.testing.assert_array_equal(ls, lse[:, :, rows])
+
+
+# ---------------------------------------------------------------- decode
+
+
+def test_decode_equals_last_causal_row_by_brute_force():
+    B, Hq, Hkv, D, cap = 2, 4, 2, 3, 6
+    lens = [4, 6]
+    kc, vc = _rand((B, Hkv, cap, D), 70), _rand((B, Hkv, cap, D), 71)
+    q = _rand((B, Hq, D), 72)
+    o, lse = decode_ref(q, kc, vc, lens, scale=0.8)
+    for b in range(B):
+        n = lens[b]
+        ob, lb = brute_force_attention(q[b : b + 1, :, None].tolist(), kc[b : b + 1, :, :n].tolist(),
+                                       vc[b : b + 1, :, :n].tolist(), causal=True, scale=0.8)
+        np.testing.assert_allclose(o[b], np.array(ob)[0, :, 0], atol=1e-14)
+        np.testing.assert_allclose(lse[b], np.array(lb)[0, :, 0], atol=1e-14)
+
+
+def test_decode_paged_equals_contiguous():
+    B, Hq, Hkv, D, bs = 3, 4, 2, 4, 4
+    lens = np.array([5, 1, 8])
+    cap = 8
+    kc, vc = _rand((B, Hkv, cap, D), 73), _rand((B, Hkv, cap, D), 74)
+    q = _rand((B, Hq, D), 75)
+    nblk = -(-lens // bs)
+    perm = np.random.Generator(np.random.PCG64(76)).permutation(int(nblk.sum()))
+    table = np.full((B, 2), -1)
+    kp = np.full((int(nblk.sum()), Hkv, bs, D), np.nan)
+    vp = np.full_like(kp, np.nan)
+    off = 0
+    for b in range(B):
+        for i in range(nblk[b]):
+            blk = perm[off]
+            off += 1
+            table[b, i] = blk
+            n = min(bs, lens[b] - i * bs)
+            kp[blk, :, :n] = kc[b, :, i * bs : i * bs + n]
+            vp[blk, :, :n] = vc[b, :, i * bs : i * bs + n]
+    o1, l1 = decode_ref(q, kc, vc, lens)
+    o2, l2 = decode_ref(q, kp, vp, lens, block_table=table, block_size=bs)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    assert np.isfinite(o2).all()
+
+
+def test_decode_empty_sequence():
+    q = _rand((2, 2, 3), 77)
+    kc = _rand((2, 1, 4, 3), 78)
+    o, lse = decode_ref(q, kc, kc, [0, 2])
+    assert np.all(o[0] == 0) and np.all(np.isneginf(lse[0]))
+    assert np.all(np.isfinite(lse[1]))
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+
+def _mismatch_vs_brute(causal=True, sq=5, sk=7, scale=0.6):
+    q, k, v = _rand((1, 4, sq, 3), 80), _rand((1, 2, sk, 3), 81), _rand((1, 2, sk, 3), 82)
+    o, _ = attention_ref(q, k, v, causal=causal, scale=scale)
+    ob, _ = _bf((q, k, v, dict(causal=causal, scale=scale)))
+    return float(np.nanmax(np.abs(o - np.array(ob))))
+
+
+def test_planted_wrong_head_mapping_is_caught(monkeypatch):
+    fake = types.SimpleNamespace(**{n: getattr(np, n) for n in dir(np) if not n.startswith("__")})
+    fake.repeat = lambda a, g, axis: np.tile(a, (1, g, 1, 1))  # head h -> kv head h % Hkv
+    monkeypatch.setattr(oatt, "np", fake)
+    assert _mismatch_vs_brute() > 1e-3
+
+
+def test_planted_dropped_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(oatt, "_default_scale", lambda d, s: 1.0)
+    assert _mismatch_vs_brute(scale=0.6) > 1e-3
+
+
+def test_planted_top_left_causal_is_caught(monkeypatch):
+    def top_left(sq, sk, causal, rows=None):
+        rows = np.arange(sq) if rows is None else np.asarray(rows)
+        return np.arange(sk)[None, :] <= rows[:, None] if causal else np.ones((rows.size, sk), bool)
+
+    monkeypatch.setattr(oatt, "allowed_mask", top_left)
+    assert _mismatch_vs_brute(sq=5, sk=7) > 1e-3
+
+
+# ---------------------------------------------------------------- plan restatement
+
+
+@pytest.mark.parametrize("args", [(16, 32, 8, 4096), (64, 32, 8, 8192), (1, 4, 4, 1), (3, 32, 1, 1000),
+                                  (2, 6, 2, 0), (128, 64, 8, 300)])
+def test_decode_plan_invariants(args):
+    B, Hq, Hkv, L = args
+    chunk, ms, G = decode_plan_ref(B, Hq, Hkv, L)
+    assert chunk % 64 == 0 and chunk >= 64
+    assert ms >= 1 and chunk * ms >= L
+    assert (Hq // Hkv) % G == 0 and G in (1, 2, 4, 8)
+    if L > 0:
+        assert chunk * (ms - 1) < L  # no split is empty at the maximum length
