@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Throughput of exact GQA attention on B200: prefill TFLOP/s and decode KV GB/s.
+
+One step is one pass of the whole hot path over synthetic inputs resident in HBM:
+
+* prefill head-sharing sweep: B=2, Hq=32, Hkv in {32, 8, 1}, Sq=Sk=2048, D=128, bf16,
+  causal -- three ``attn_fwd`` calls (one tensor-core kernel each);
+* paged GQA decode: B=64, Hq=32, Hkv=8, D=128, block 16, lengths U[512, 8192], pool
+  permuted -- one ``attn_decode`` call (split kernel + combine kernel);
+* contiguous GQA decode: B=16, Hq=32, Hkv=8, D=128, capacity 4096, lengths
+  U[1024, 4096] -- one ``attn_decode`` call.
+
+L2 (126 MB) is flushed with a 256 MiB write before every call; each call is timed
+with CUDA events on the launching stream.  ``value`` is the prefill throughput
+(algorithmic FLOPs = 4*D*B*Hq*S(S+1)/2 per call, unmasked pairs only) summed over
+all ranks; the decode numbers (valid-token K/V bytes per call) are in ``decode``.
+Under torchrun every rank runs an independent replica (the path needs no exchange).
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "GQA prefill TFLOP/s & decode KV GB/s on 1 B200, as % of roofline"
+PREFILL = dict(B=2, Hq=32, S=2048, D=128, hkvs=(32, 8, 1))
+PAGED = dict(B=64, Hq=32, Hkv=8, D=128, bs=16, lo=512, hi=8192)
+CONTIG = dict(B=16, Hq=32, Hkv=8, D=128, cap=4096, lo=1024, hi=4096)
+FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def prefill_flops(B, Hq, S, D):
+    return 4.0 * D * B * Hq * S * (S + 1) / 2.0
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.flush()
+        with open(self.out.name) as f:
+            lines = [ln.strip() for ln in f if ln.strip()]
+        os.unlink(self.out.name)
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                maxs.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(name)
+        if not sms:
+            return None
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_init():
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ oracle timing
+
+
+def oracle_prefill_sample(target_s: float):
+    """Time the fp64 oracle on whole query heads of the GQA (Hkv=8) S=2048 causal case."""
+    import numpy as np
+
+    from exact_attention_137_b200.workloads import prefill_inputs, to_f64
+    from oracle import attention_ref
+
+    B, Hq, S, D = 1, 32, PREFILL["S"], PREFILL["D"]
+    x = prefill_inputs(B, Hq, 8, S, S, D, dtype="bf16", seed=0)
+    q, k, v = to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"])
+    g = Hq // 8
+    t0 = time.perf_counter()
+    attention_ref(q[:, :1], k[:, :1], v[:, :1], causal=True)
+    t1 = time.perf_counter() - t0
+    nh = int(max(1, min(Hq, round(target_s / max(t1, 1e-3)))))
+    nkv = -(-nh // g)
+    t0 = time.perf_counter()
+    attention_ref(q[:, :nh], k[:, :nkv], v[:, :nkv], causal=True)
+    dt = time.perf_counter() - t0
+    flops = prefill_flops(1, nh, S, D)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"b=0, query heads 0..{nh - 1} (all {S} rows) of the Hkv=8 S={S} D={D} causal case; "
+                      f"{dt:.1f} s; numpy fp64 with full score matrices"}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle, timed on the host, on a bounded sample per step."""
+    if rank != 0:
+        return
+    import numpy as np
+
+    from exact_attention_137_b200.workloads import prefill_inputs, to_f64
+    from oracle import attention_rows_ref
+
+    S, D = PREFILL["S"], PREFILL["D"]
+    inputs = []
+    for hkv in PREFILL["hkvs"]:
+        x = prefill_inputs(1, PREFILL["Hq"], hkv, S, S, D, dtype="bf16", seed=0)
+        g = PREFILL["Hq"] // hkv
+        # one query head (and its K/V head) per variant, the last 64 rows
+        inputs.append((to_f64(x["q"][:, :1]), to_f64(x["k"][:, :1]), to_f64(x["v"][:, :1])))
+    rows = np.arange(S - 64, S)
+    step_flops = sum(4.0 * D * float(np.sum(rows + 1)) for _ in inputs)
+
+    def step():
+        for q, k, v in inputs:
+            attention_rows_ref(q, k, v, causal=True, rows=rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = step_flops * args.steps / dt / 1e12
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"per step: one query head of each Hkv in {PREFILL['hkvs']} variant (B=2, Hq=32, S={S}, D={D}, "
+              f"causal), last 64 query rows, each over its full visible key range")
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "prefill head-sharing sweep B=2 Hq=32 Hkv in {32,8,1} S=2048 D=128 causal "
+                                   "(row sample)", "oracle": "numpy fp64, full score matrix per head"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+
+
+def run_ours(args, rank, world, local):
+    import torch
+
+    from exact_attention_137_b200 import attn_decode, attn_fwd, decode_workspace, device_status, load
+    from exact_attention_137_b200.workloads import decode_contiguous_inputs, decode_paged_inputs, prefill_inputs
+
+    load()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    seed = rank
+    peaks, peak_src = load_peaks()
+    P = PREFILL
+    pre = []
+    for hkv in P["hkvs"]:
+        x = prefill_inputs(P["B"], P["Hq"], hkv, P["S"], P["S"], P["D"], dtype="bf16", seed=seed)
+        q, k, v = x["q"].to(dev), x["k"].to(dev), x["v"].to(dev)
+        pre.append(dict(hkv=hkv, q=q, k=k, v=v, o=torch.empty_like(q),
+                        lse=torch.empty(q.shape[:3], device=dev, dtype=torch.float32), host=x))
+    fl_call = prefill_flops(P["B"], P["Hq"], P["S"], P["D"])
+
+    def decode_case(x, spec):
+        g = {kk: (vv.to(dev) if isinstance(vv, torch.Tensor) else vv) for kk, vv in x.items()}
+        g["ws"] = decode_workspace(spec["B"], spec["Hq"], spec["Hkv"], spec["D"], x["max_seqlen"], dev)
+        g["o"] = torch.empty_like(g["q"])
+        g["lse"] = torch.empty(g["q"].shape[:2], device=dev, dtype=torch.float32)
+        lens = x["seqlens"].numpy().astype("int64")
+        kv = float(lens.sum()) * spec["Hkv"] * spec["D"] * 2 * 2
+        io = g["q"].numel() * 2 * 2 + g["lse"].numel() * 4 + lens.size * 4
+        if x["block_table"] is not None:
+            io += float(((lens + spec["bs"] - 1) // spec["bs"]).sum()) * 4
+        g["bytes"] = kv + io
+        g["kv_bytes"] = kv
+        return g
+
+    S = PAGED
+    paged = decode_case(decode_paged_inputs(S["B"], S["Hq"], S["Hkv"], S["D"], S["bs"], S["lo"], S["hi"], seed=seed),
+                        S)
+    C = CONTIG
+    contig = decode_case(decode_contiguous_inputs(C["B"], C["Hq"], C["Hkv"], C["D"], C["cap"], C["lo"], C["hi"],
+                                                  seed=seed), dict(C, bs=C["cap"]))
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def run_prefill(c):
+        attn_fwd(c["q"], c["k"], c["v"], causal=True, o=c["o"], lse=c["lse"])
+
+    def run_decode(g):
+        attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=g["max_seqlen"],
+                    block_table=g["block_table"], workspace=g["ws"], o=g["o"], lse=g["lse"])
+
+    calls = [("prefill_hkv%d" % c["hkv"], (lambda c=c: run_prefill(c))) for c in pre]
+    calls += [("decode_paged", lambda: run_decode(paged)), ("decode_contiguous", lambda: run_decode(contig))]
+    launches_per_step = len(pre) * 1 + 2 * 2
+    nev = len(calls)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nev)]
+          for _ in range(args.steps)]
+
+    def step(i=None):
+        for ci, (_, fn) in enumerate(calls):
+            flush.fill_(float(ci))
+            if i is not None:
+                ev[i][ci][0].record(stream)
+            fn()
+            if i is not None:
+                ev[i][ci][1].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert device_status(clear=True) == 0
+
+    clocks = ClockSampler(torch.cuda.current_device() if world == 1 else local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(i)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    status = device_status(clear=True)
+    total_ms = t_start.elapsed_time(t_end)
+    per_call = {name: sum(ev[i][ci][0].elapsed_time(ev[i][ci][1]) for i in range(args.steps)) / args.steps
+                for ci, (name, _) in enumerate(calls)}
+    pre_ms = sum(per_call["prefill_hkv%d" % c["hkv"]] for c in pre)
+    pre_ms_max = max_over_ranks(pre_ms, world)
+    total_ms_max = max_over_ranks(total_ms, world)
+    value = world * len(pre) * fl_call / (pre_ms_max * 1e-3) / 1e12
+
+    # e2e: host (pinned) inputs -> device -> attn_fwd -> host outputs, through the public API.
+    e2e_steps = min(args.steps, 10)
+    hostbuf = []
+    for c in pre:
+        h = {n: c["host"][n].pin_memory() for n in ("q", "k", "v")}
+        h["o"] = torch.empty(c["q"].shape, dtype=torch.bfloat16).pin_memory()
+        h["lse"] = torch.empty(c["lse"].shape, dtype=torch.float32).pin_memory()
+        hostbuf.append(h)
+    h2d = sum(sum(h[n].numel() * h[n].element_size() for n in ("q", "k", "v")) for h in hostbuf)
+    d2h = sum(h["o"].numel() * 2 + h["lse"].numel() * 4 for h in hostbuf)
+
+    def e2e_step():
+        for c, h in zip(pre, hostbuf):
+            c["q"].copy_(h["q"], non_blocking=True)
+            c["k"].copy_(h["k"], non_blocking=True)
+            c["v"].copy_(h["v"], non_blocking=True)
+            run_prefill(c)
+            h["o"].copy_(c["o"], non_blocking=True)
+            h["lse"].copy_(c["lse"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
+    e2e_value = world * len(pre) * fl_call / (e2e_ms * 1e-3) / 1e12
+
+    hbm = peaks["hbm_gbs"]
+    tf_peak = peaks["bf16_tflops"]
+    per_launch_ms = pre_ms / len(pre)
+    achieved_tf = fl_call / (per_launch_ms * 1e-3) / 1e12
+
+    def dec_obj(name, g, spec_name):
+        ms = max_over_ranks(per_call[name], world)
+        gbs = g["bytes"] / (ms * 1e-3) / 1e9
+        return {"workload": spec_name, "ms": ms, "GB/s": gbs, "kv_bytes": g["kv_bytes"], "bytes": g["bytes"],
+                "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "kernels": ["split", "combine"]}
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": total_ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "prefill head-sharing sweep B=2 Hq=32 Hkv in {32,8,1} Sq=Sk=2048 D=128 bf16 causal "
+                               "(value); decode paged B=64 and contiguous B=16 (decode)",
+                   "l2": "flushed by a 256 MiB write before every timed call",
+                   "prefill_flops_per_call": fl_call, "prefill_ms_per_call": {c["hkv"]: per_call["prefill_hkv%d" % c["hkv"]] for c in pre},
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "roofline": {"bound": "tensor", "kernel": "attn::tc::fwd_tc_kernel<128>", "achieved": achieved_tf,
+                     "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved_tf / tf_peak, "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst)"},
+        "decode": {"paged": dec_obj("decode_paged", paged, "B=64 Hq=32 Hkv=8 D=128 block 16 len U[512,8192]"),
+                   "contiguous": dec_obj("decode_contiguous", contig,
+                                         "B=16 Hq=32 Hkv=8 D=128 cap 4096 len U[1024,4096]")},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "prefill sweep with q/k/v copied from pinned host memory and O/LSE copied back each step"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "device_status": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = oracle_prefill_sample(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_init()
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,245 @@
+"""ctypes binding to ``libattn137.so``: argument marshalling only.
+
+Every step of the attention path runs in the library's CUDA kernels; this module
+checks tensor shapes/dtypes, allocates outputs with torch, and passes raw device
+pointers and the current CUDA stream.  There is no fallback: if the library is
+missing, every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn137.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "attn.h")
+
+ATTN_OK = 0
+ATTN_ERR_ARG = 1
+ATTN_ERR_HEADS = 2
+ATTN_ERR_UNSUPPORTED = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_DEVICE = 5
+ATTN_ERR_WORKSPACE = 6
+ATTN_BF16 = 0
+ATTN_F32 = 1
+ATTN_DEV_WAIT_TIMEOUT = 1
+ATTN_DEV_BAD_BLOCK = 2
+ATTN_DEV_BAD_SEQLEN = 4
+
+_c_int, _c_float, _vp, _size_t, _ll, _ull = (ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t,
+                                           ctypes.c_longlong, ctypes.c_ulonglong)
+_ip = ctypes.POINTER(ctypes.c_int)
+
+_SIGS = {
+    "attn_error_string": (ctypes.c_char_p, [_c_int]),
+    "attn_abi_version": (_c_int, []),
+    "attn_fwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                          _c_int, _c_int, _vp]),
+    "attn_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                             _c_int, _c_float, _vp, _size_t, _vp, _vp, _c_int, _vp]),
+    "attn_decode_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "attn_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _ip, _ip, _ip]),
+    "attn_decode_check": (_c_int, [_vp, _vp]),
+    "attn_device_status": (_c_int, [_c_int, _vp]),
+    "attn_selftest_wait_timeout": (_c_int, [_ull, _vp]),
+    "attn_kv_cache_bytes": (_size_t, [_c_int, _c_int, _c_int, _ll, _c_int, _c_int]),
+    "attn_paged_pool_blocks": (_ll, [_ip, _c_int, _c_int]),
+    "attn_paged_pool_bytes": (_size_t, [_ll, _c_int, _c_int, _c_int, _c_int]),
+}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {error_string(status) if _lib else status} (status {status})")
+
+
+def load() -> ctypes.CDLL:
+    """Load the library once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m exact_attention_137_b200.build` (no fallback exists)")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/attn.h."""
+    with open(HEADER_PATH, encoding="utf-8") as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text, flags=re.M)
+
+
+def error_string(status: int) -> str:
+    return load().attn_error_string(status).decode()
+
+
+def _check(status: int, where: str):
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _stream_ptr(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ prefill
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, lse=None,
+             return_lse: bool = True, stream=None):
+    """Attention forward: ``q [B,Hq,Sq,D]``, ``k``/``v`` ``[B,Hkv,Sk,D]`` on the GPU.
+
+    Returns ``(o, lse)`` (``lse`` is ``None`` when ``return_lse`` is false and none
+    was passed).
+    """
+    lib = load()
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, S, D]")
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k.shape
+    if v.shape != k.shape or k.shape[0] != B or k.shape[3] != D:
+        raise ValueError("shape mismatch between q, k and v")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share a dtype")
+    for t in (q, k, v):
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, sc,
+                      1 if causal else 0, _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(st, "attn_fwd")
+    return o, lse
+
+
+# ------------------------------------------------------------------ decode
+
+
+def decode_plan(B: int, Hq: int, Hkv: int, max_seqlen: int):
+    lib = load()
+    c, m, g = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(lib.attn_decode_plan(B, Hq, Hkv, max_seqlen, ctypes.byref(c), ctypes.byref(m), ctypes.byref(g)),
+           "attn_decode_plan")
+    return c.value, m.value, g.value
+
+
+def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, max_seqlen: int) -> int:
+    return int(load().attn_decode_workspace_bytes(B, Hq, Hkv, D, max_seqlen))
+
+
+def decode_workspace(B, Hq, Hkv, D, max_seqlen, device) -> torch.Tensor:
+    """Zero-filled workspace of the required size (torch allocations are 256-byte aligned)."""
+    return torch.zeros(decode_workspace_bytes(B, Hq, Hkv, D, max_seqlen), dtype=torch.uint8, device=device)
+
+
+def attn_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None, block_size: int | None = None,
+                scale: float | None = None, workspace=None, o=None, lse=None, return_lse: bool = True,
+                stream=None):
+    """Single-token decode.  ``q [B,Hq,D]`` bf16; ``seqlens [B]`` int32 on the GPU.
+
+    Paged: ``k_cache``/``v_cache`` ``[num_blocks,Hkv,block_size,D]`` and
+    ``block_table [B,max_blocks]`` int32.  Contiguous: ``[B,Hkv,cap,D]`` and
+    ``block_table=None``.  Returns ``(o, lse)``.
+    """
+    lib = load()
+    if q.dim() != 3:
+        raise ValueError("q must be [B, Hq, D]")
+    B, Hq, D = q.shape
+    if k_cache.dim() != 4 or v_cache.shape != k_cache.shape or k_cache.shape[3] != D:
+        raise ValueError("k_cache/v_cache must share a 4-D shape ending in D")
+    Hkv = k_cache.shape[1]
+    if block_table is None:
+        if k_cache.shape[0] != B:
+            raise ValueError("contiguous cache must be [B, Hkv, cap, D]")
+        bs = k_cache.shape[2]
+        max_blocks, num_blocks = 1, B
+    else:
+        if block_table.dtype != torch.int32 or block_table.dim() != 2 or block_table.shape[0] != B:
+            raise ValueError("block_table must be int32 [B, max_blocks]")
+        bs = k_cache.shape[2] if block_size is None else int(block_size)
+        if bs != k_cache.shape[2]:
+            raise ValueError("block_size does not match the pool")
+        max_blocks, num_blocks = block_table.shape[1], k_cache.shape[0]
+        if not block_table.is_contiguous():
+            raise ValueError("block_table must be contiguous")
+    if seqlens.dtype != torch.int32 or seqlens.numel() != B or not seqlens.is_cuda:
+        raise ValueError("seqlens must be a CUDA int32 tensor of B entries")
+    for t in (q, k_cache, v_cache, seqlens):
+        if not t.is_contiguous():
+            raise ValueError("inputs must be contiguous")
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, D, max_seqlen, q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(block_table), bs, max_blocks,
+                         num_blocks, int(max_seqlen), B, Hq, Hkv, D, sc, _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _ptr(o), _ptr(lse), _dtype_code(q),
+                         ctypes.c_void_p(_stream_ptr(stream)))
+    _check(st, "attn_decode")
+    return o, lse
+
+
+def decode_check(workspace, stream=None) -> int:
+    return int(load().attn_decode_check(_ptr(workspace), ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def device_status(clear: bool = False, stream=None) -> int:
+    return int(load().attn_device_status(1 if clear else 0, ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def selftest_wait_timeout(timeout_ns: int, stream=None) -> int:
+    return int(load().attn_selftest_wait_timeout(int(timeout_ns), ctypes.c_void_p(_stream_ptr(stream))))
+
+
+# ------------------------------------------------------------------ KV-cache sizing (host only)
+
+
+def kv_cache_bytes(layers: int, kv_heads: int, head_dim: int, tokens: int, batch: int, elem_bytes: int) -> int:
+    return int(load().attn_kv_cache_bytes(layers, kv_heads, head_dim, tokens, batch, elem_bytes))
+
+
+def paged_pool_blocks(seqlens, block_size: int) -> int:
+    arr = (ctypes.c_int * len(seqlens))(*[int(x) for x in seqlens])
+    return int(load().attn_paged_pool_blocks(arr, len(seqlens), block_size))
+
+
+def paged_pool_bytes(num_blocks: int, kv_heads: int, block_size: int, head_dim: int, elem_bytes: int) -> int:
+    return int(load().attn_paged_pool_bytes(num_blocks, kv_heads, block_size, head_dim, elem_bytes))

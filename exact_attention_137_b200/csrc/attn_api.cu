@@ -1,0 +1,393 @@
+// Host side of the C ABI declared in include/attn.h: argument validation, the split-KV
+// plan, TMA descriptor encoding and kernel launches.  One translation unit so that the
+// device status word is a single symbol per device.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_simt.cuh"
+#include "prefill_tc.cuh"
+
+namespace {
+
+using attn::tc::BM;
+using attn::tc::BN;
+
+constexpr int kAbiVersion = 1;
+constexpr int kDecodeTargetCtas = 2368;
+constexpr size_t kWsHeader = 256;
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+// ------------------------------------------------------------------ tensor maps
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [heads, rows, D] bf16 viewed as 3-D (D, rows, heads); 64-column x 128-row boxes with the
+// 128-byte swizzle that the tcgen05 shared-memory descriptors expect.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, int D, int rows, long long heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)heads};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)rows * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)BM, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Per-device one-time kernel attribute setup.
+template <typename F>
+cudaError_t set_smem_once(F* kernel, int bytes, int key) {
+  static bool done[64][8] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || key < 0 || key >= 8) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lk(mu);
+  if (done[dev][key]) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done[dev][key] = true;
+  return e;
+}
+
+__global__ void fill_empty_rows_kernel(float* lse, size_t n) {
+  size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < n) lse[i] = -INFINITY;
+}
+
+template <int D>
+int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Sq, int Sk, float scale, int causal, cudaStream_t st) {
+  using Lay = attn::tc::Layout<D>;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bf16(&tq, q, D, Sq, (long long)B * Hq) || !make_tmap_bf16(&tk, k, D, Sk, (long long)B * Hkv) ||
+      !make_tmap_bf16(&tv, v, D, Sk, (long long)B * Hkv))
+    return ATTN_ERR_CUDA;
+  attn::tc::Params p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.scale_log2 = scale * attn::kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.nq = (int)cdiv(Sq, BM);
+  const int g = Hq / Hkv;
+  p.pairs = g / 2;
+  const long long items_a = (long long)p.nq * B * Hkv * p.pairs;
+  p.npq = (g & 1) ? (int)cdiv(p.nq, 2) : 0;
+  const long long items_b = (long long)p.npq * B * Hkv;
+  if (items_a + items_b > INT_MAX) return ATTN_ERR_UNSUPPORTED;
+  p.items_a = (int)items_a;
+  const int grid = (int)(items_a + items_b);
+  auto kern = attn::tc::fwd_tc_kernel<D>;
+  cudaError_t e = set_smem_once(kern, Lay::kAlloc, D == 64 ? 0 : 1);
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  kern<<<grid, attn::tc::kThreads, Lay::kAlloc, st>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <typename T, int D>
+int launch_fwd_simt(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                    int Hkv, int Sq, int Sk, float scale, int causal, cudaStream_t st) {
+  dim3 grid((unsigned)cdiv(Sq, attn::simt::kRowsPerBlock), (unsigned)(B * Hq));
+  if (grid.y > 65535u) return ATTN_ERR_UNSUPPORTED;
+  attn::simt::fwd_simt_kernel<T, D><<<grid, attn::simt::kRowsPerBlock * 32, 0, st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o), lse,
+      Hq, Hkv, Sq, Sk, scale * attn::kLog2e, causal ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+struct DecodePlan {
+  int chunk, max_splits, G;
+};
+
+bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_seqlen < 0 || Hq % Hkv) return false;
+  const int g = Hq / Hkv;
+  int G = 1;
+  for (int cand : {8, 4, 2, 1})
+    if (g % cand == 0) {
+      G = cand;
+      break;
+    }
+  const long long streams = (long long)B * Hkv * (g / G);
+  long long splits = cdiv(kDecodeTargetCtas, streams);
+  const long long cap = std::max(1LL, cdiv(max_seqlen, 256));
+  splits = std::max(1LL, std::min(splits, cap));
+  const long long per = cdiv(std::max(max_seqlen, 1), splits);
+  const long long chunk = std::max(64LL, 64 * cdiv(per, 64));
+  out->chunk = (int)chunk;
+  out->max_splits = (int)std::max(1LL, cdiv(max_seqlen, chunk));
+  out->G = G;
+  return true;
+}
+
+size_t ws_lse_bytes(int B, int Hq, int ms) {
+  size_t n = (size_t)B * Hq * ms * sizeof(float);
+  return (n + 255) & ~size_t(255);
+}
+
+template <int D, int G>
+int launch_decode_split(const attn::dec::Params& p, cudaStream_t st) {
+  using Lay = attn::dec::Layout<D>;
+  auto kern = attn::dec::decode_split_kernel<D, G>;
+  const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3);
+  static bool done[64][8] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (!done[dev][key]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::kBytes) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+      done[dev][key] = true;
+    }
+  }
+  dim3 grid((unsigned)p.max_splits, (unsigned)(p.Hkv * p.nsub), (unsigned)p.B);
+  kern<<<grid, attn::dec::kThreads, Lay::kBytes, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  attn::dec::decode_combine_kernel<D><<<(unsigned)(p.B * p.Hq), D, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D>
+int dispatch_decode_g(const attn::dec::Params& p, int G, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_split<D, 1>(p, st);
+    case 2: return launch_decode_split<D, 2>(p, st);
+    case 4: return launch_decode_split<D, 4>(p, st);
+    case 8: return launch_decode_split<D, 8>(p, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = attn::smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    attn::mbar_init(b, 1);
+    abort_flag = 0;
+    attn::fence_barrier_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on this barrier: the wait must give up and report it.
+  attn::mbar_wait(b, 0, &abort_flag, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_error_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_ARG: return "invalid argument";
+    case ATTN_ERR_HEADS: return "query heads are not a multiple of kv heads";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported head dim, dtype or shape";
+    case ATTN_ERR_CUDA: return "CUDA call failed";
+    case ATTN_ERR_DEVICE: return "a kernel flagged a device-side error";
+    case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    default: return "unknown status";
+  }
+}
+
+int attn_abi_version(void) { return kAbiVersion; }
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
+             int Sk, int D, float scale, int causal, int dtype, void* stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || !std::isfinite(scale)) return ATTN_ERR_ARG;
+  // q/o may be NULL only when Sq == 0, k/v only when Sk == 0 (nothing is read or written).
+  if ((Sq > 0 && (!q || !o)) || (Sk > 0 && (!k || !v))) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > INT_MAX / 2 || (long long)Sq * D > INT_MAX || (long long)Sk * D > INT_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  if (Sq == 0) return ATTN_OK;
+  const size_t elem = dtype == ATTN_BF16 ? 2 : 4;
+  if (Sk == 0) {
+    const size_t rows = (size_t)B * Hq * Sq;
+    if (cudaMemsetAsync(o, 0, rows * D * elem, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_empty_rows_kernel<<<(unsigned)cdiv((long long)rows, 256), 256, 0, st>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (dtype == ATTN_BF16) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ARG;
+    return D == 64 ? launch_fwd_tc<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st)
+                   : launch_fwd_tc<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st);
+  }
+  return D == 64 ? launch_fwd_simt<float, 64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st)
+                 : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st);
+}
+
+int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int* chunk_tokens, int* max_splits,
+                     int* heads_per_cta) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_seqlen < 0) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  DecodePlan pl;
+  if (!decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return ATTN_ERR_ARG;
+  if (chunk_tokens) *chunk_tokens = pl.chunk;
+  if (max_splits) *max_splits = pl.max_splits;
+  if (heads_per_cta) *heads_per_cta = pl.G;
+  return ATTN_OK;
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen) {
+  DecodePlan pl;
+  if (D <= 0 || !decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return 0;
+  return kWsHeader + ws_lse_bytes(B, Hq, pl.max_splits) + (size_t)B * Hq * pl.max_splits * D * sizeof(float);
+}
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
+                int block_size, int max_blocks, int num_blocks, int max_seqlen, int B, int Hq, int Hkv, int D,
+                float scale, void* workspace, size_t workspace_bytes, void* o, float* lse, int dtype,
+                void* stream) {
+  if (!q || !k_cache || !v_cache || !seqlens || !o) return ATTN_ERR_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || block_size <= 0 || max_seqlen < 0 || !std::isfinite(scale))
+    return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (block_table) {
+    if (max_blocks <= 0 || num_blocks <= 0) return ATTN_ERR_ARG;
+  } else {
+    num_blocks = B;  // a dense cache is the paged layout with block b = sequence b
+    max_blocks = 1;
+  }
+  if (B > 65535 || (long long)Hkv * Hq > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o)) return ATTN_ERR_ARG;
+  DecodePlan pl;
+  if (!decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return ATTN_ERR_ARG;
+  const size_t need = attn_decode_workspace_bytes(B, Hq, Hkv, D, max_seqlen);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < need)
+    return ATTN_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  attn::dec::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
+  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.seqlens = seqlens;
+  p.block_table = block_table;
+  p.block_size = block_size;
+  p.max_blocks = max_blocks;
+  p.num_blocks = num_blocks;
+  p.max_seqlen = max_seqlen;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.chunk = pl.chunk;
+  p.max_splits = pl.max_splits;
+  p.nsub = (Hq / Hkv) / pl.G;
+  p.scale_log2 = scale * attn::kLog2e;
+  p.ws_err = reinterpret_cast<unsigned int*>(ws);
+  p.ws_lse = reinterpret_cast<float*>(ws + kWsHeader);
+  p.ws_o = reinterpret_cast<float*>(ws + kWsHeader + ws_lse_bytes(B, Hq, pl.max_splits));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  cudaStream_t st = as_stream(stream);
+  return D == 64 ? dispatch_decode_g<64>(p, pl.G, st) : dispatch_decode_g<128>(p, pl.G, st);
+}
+
+int attn_decode_check(void* workspace, void* stream) {
+  if (!workspace) return ATTN_ERR_WORKSPACE;
+  cudaStream_t st = as_stream(stream);
+  unsigned int word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_ERR_DEVICE;
+  }
+  return ATTN_OK;
+}
+
+int attn_device_status(int clear, void* stream) {
+  cudaStream_t st = as_stream(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_status, sizeof(v)) != cudaSuccess) return -1;
+  if (clear) {
+    const unsigned int z = 0;
+    if (cudaMemcpyToSymbol(attn::g_status, &z, sizeof(z)) != cudaSuccess) return -1;
+  }
+  return (int)v;
+}
+
+int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
+  if (timeout_ns > 1000000000ull) timeout_ns = 1000000000ull;
+  selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_kv_cache_bytes(int layers, int kv_heads, int head_dim, long long tokens, int batch, int elem_bytes) {
+  if (layers < 0 || kv_heads < 0 || head_dim < 0 || tokens < 0 || batch < 0 || elem_bytes < 0) return 0;
+  unsigned __int128 n = 2;
+  n *= (unsigned)layers;
+  n *= (unsigned)kv_heads;
+  n *= (unsigned)head_dim;
+  n *= (unsigned long long)tokens;
+  n *= (unsigned)batch;
+  n *= (unsigned)elem_bytes;
+  if (n > (unsigned __int128)SIZE_MAX) return 0;
+  return (size_t)n;
+}
+
+long long attn_paged_pool_blocks(const int* seqlens_host, int B, int block_size) {
+  if (!seqlens_host || B < 0 || block_size <= 0) return -1;
+  long long total = 0;
+  for (int b = 0; b < B; ++b) {
+    if (seqlens_host[b] < 0) return -1;
+    total += cdiv(seqlens_host[b], block_size);
+  }
+  return total;
+}
+
+size_t attn_paged_pool_bytes(long long num_blocks, int kv_heads, int block_size, int head_dim, int elem_bytes) {
+  if (num_blocks < 0 || kv_heads < 0 || block_size < 0 || head_dim < 0 || elem_bytes < 0) return 0;
+  unsigned __int128 n = (unsigned long long)num_blocks;
+  n *= (unsigned)kv_heads;
+  n *= (unsigned)block_size;
+  n *= (unsigned)head_dim;
+  n *= (unsigned)elem_bytes;
+  if (n > (unsigned __int128)SIZE_MAX) return 0;
+  return (size_t)n;
+}
+
+}  // extern "C"

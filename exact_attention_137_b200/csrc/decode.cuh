@@ -1,0 +1,369 @@
+// Single-token decode over a contiguous or paged KV cache: split-KV partials plus an
+// LSE-weighted combine pass.
+//
+// The KV cache is read once from HBM, which bounds the step (CSDN «注意力变体深挖» §一
+// and §七: decoding is memory-bound on KV reads).  Design for sm_100a:
+//
+//  * grid (split, kv head x head-subgroup, batch).  A CTA reads the K/V of one KV head
+//    for one chunk of tokens and serves the G query heads of its subgroup from that
+//    single read (GQA: the group's heads share each K/V row).
+//  * warp 4 streams the chunk through a 4-stage shared-memory ring with cp.async.bulk:
+//    every run of tokens that is contiguous in the cache (one page of a paged pool, or
+//    the whole stage in a dense cache) is one bulk copy.  The page ids come from the
+//    block table (gocoding §5), prefetched 32 pages ahead into the producer's lanes.
+//  * warps 0-3 compute.  D/8 lanes cover one 128-bit slice each of a token's row;
+//    per step each lane forms the partial dot products of D/8 (token, head) pairs and a
+//    reduce-scatter across the lane group leaves one complete score per lane.  Online
+//    softmax per head (log2 domain, ex2), then the value rows are accumulated in fp32.
+//  * each split writes its normalised partial output and its LSE; the combine kernel
+//    merges the splits of a (sequence, head) with weights exp(lse_s - LSE), the same
+//    two-way merge as the pages' online softmax, applied across splits.
+#pragma once
+
+#include "common.cuh"
+
+namespace attn {
+namespace dec {
+
+constexpr int kStageTokens = 32;
+constexpr int kStages = 4;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* kc;
+  const __nv_bfloat16* vc;
+  const int* seqlens;
+  const int* block_table;  // nullptr: contiguous cache
+  int block_size, max_blocks, num_blocks, max_seqlen;
+  int B, Hq, Hkv;
+  int chunk, max_splits, nsub;
+  float scale_log2;
+  float* ws_o;    // [B, Hq, max_splits, D]
+  float* ws_lse;  // [B, Hq, max_splits]
+  unsigned int* ws_err;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+template <int D>
+struct Layout {
+  static constexpr int kRow = D * 2;
+  static constexpr int kStageBytes = kStageTokens * kRow;  // K (or V) bytes of one stage
+  static constexpr int kK = 0;
+  static constexpr int kV = kStages * kStageBytes;
+  static constexpr int kBar = 2 * kStages * kStageBytes;
+  static constexpr int kMisc = kBar + 2 * kStages * 8;
+  static constexpr int kBytes = kMisc + 16;
+};
+
+__device__ __forceinline__ void flag_error(const Params& p, unsigned int f) {
+  atomicOr(p.ws_err, f);
+  raise_status(f);
+}
+
+// Valid length of sequence b after the device-side bound checks.
+__device__ __forceinline__ int checked_len(const Params& p, int b, bool report) {
+  int len = p.seqlens[b];
+  const long long cap = p.block_table ? (long long)p.max_blocks * p.block_size : (long long)p.block_size;
+  long long lim = p.max_seqlen < cap ? p.max_seqlen : cap;
+  if (len < 0 || len > lim) {
+    if (report) flag_error(p, ATTN_DEV_BAD_SEQLEN);
+    len = len < 0 ? 0 : (int)lim;
+  }
+  return len;
+}
+
+__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
+  f[0] = bf16lo(w.x);
+  f[1] = bf16hi(w.x);
+  f[2] = bf16lo(w.y);
+  f[3] = bf16hi(w.y);
+  f[4] = bf16lo(w.z);
+  f[5] = bf16hi(w.z);
+  f[6] = bf16lo(w.w);
+  f[7] = bf16hi(w.w);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// Recursive-halving reduce-scatter over the LPT lanes of a group: on return lane j of
+// the group holds in vals[0] the group-wide sum of the original vals[j].
+template <int LPT>
+__device__ __forceinline__ float reduce_scatter(float (&vals)[LPT], int j) {
+#pragma unroll
+  for (int off = LPT / 2, cnt = LPT / 2; off > 0; off >>= 1, cnt >>= 1) {
+    const bool upper = (j & off) != 0;
+#pragma unroll
+    for (int i = 0; i < cnt; ++i) {
+      const float send = upper ? vals[i] : vals[i + cnt];
+      const float keep = upper ? vals[i + cnt] : vals[i];
+      vals[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return vals[0];
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) {
+  constexpr int LPT = D / 8;       // lanes per token row (16 bytes each)
+  constexpr int TOK = LPT / G;     // tokens per lane group per step
+  constexpr int GPW = 32 / LPT;    // lane groups per warp
+  constexpr int TPW = GPW * TOK;   // tokens per warp step (= 32 / G)
+  constexpr int UNITS = kStageTokens / TPW;  // warp steps per stage (= G)
+  static_assert(G <= LPT && TOK * G == LPT, "heads per CTA must divide the lanes per token");
+  using L = Layout<D>;
+
+  extern __shared__ __align__(128) uint8_t smem[];
+  const uint32_t sbase = smem_u32(smem);
+  auto full_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * s; };
+  auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (kStages + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
+
+  const int b = blockIdx.z;
+  const int split = blockIdx.x;
+  const int len = checked_len(p, b, split == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+  const int nsplit = (len + p.chunk - 1) / p.chunk;
+  if (split >= nsplit) return;
+  const int t0 = split * p.chunk;
+  const int t1 = min(len, t0 + p.chunk);
+  const int niters = (t1 - t0 + kStageTokens - 1) / kStageTokens;
+  const int kvh = blockIdx.y / p.nsub;
+  const int sub = blockIdx.y - kvh * p.nsub;
+  const int g = p.Hq / p.Hkv;
+  const int h0 = kvh * g + sub * G;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ bulk-copy producer
+    const int bs = p.block_size;
+    const bool paged = p.block_table != nullptr;
+    const int* table = paged ? p.block_table + (size_t)b * p.max_blocks : nullptr;
+    auto load_id = [&](int page) -> int {
+      return (paged && page < p.max_blocks) ? __ldg(table + page) : -1;
+    };
+    int cur_first = t0 / bs;
+    int nxt_first = cur_first + 32;
+    int cur_id = load_id(cur_first + lane);
+    int nxt_id = load_id(nxt_first + lane);
+    int last_fill[kStages];
+    for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+    for (int it = 0; it < niters; ++it) {
+      const int s = it % kStages;
+      const int f = it / kStages;
+      if (f > 0) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), (f - 1) & 1, abort_flag));
+        if (!ok) break;
+      }
+      const int a = t0 + it * kStageTokens;
+      const int e = min(t1, a + kStageTokens);
+      const uint32_t dk = sbase + L::kK + s * L::kStageBytes;
+      const uint32_t dv = sbase + L::kV + s * L::kStageBytes;
+      for (int tok = a; tok < e;) {
+        const int page = tok / bs;
+        const int slot = tok - page * bs;
+        const int run = min(bs - slot, e - tok);
+        while (page >= cur_first + 32) {
+          cur_id = nxt_id;
+          cur_first = nxt_first;
+          nxt_first += 32;
+          nxt_id = load_id(nxt_first + lane);
+        }
+        const int blk = paged ? __shfl_sync(0xffffffffu, cur_id, page - cur_first) : b;
+        if (lane == 0) {
+          if (blk < 0 || blk >= p.num_blocks) {
+            flag_error(p, ATTN_DEV_BAD_BLOCK);
+          } else {
+            const size_t off = (((size_t)blk * p.Hkv + kvh) * (size_t)bs + slot) * D;
+            const uint32_t bytes = (uint32_t)run * L::kRow;
+            const uint32_t dst = (uint32_t)(tok - a) * L::kRow;
+            mbar_expect_tx(full_bar(s), 2u * bytes);
+            bulk_load(dk + dst, p.kc + off, bytes, full_bar(s));
+            bulk_load(dv + dst, p.vc + off, bytes, full_bar(s));
+          }
+        }
+        tok += run;
+      }
+      if (lane == 0) mbar_arrive(full_bar(s));
+      last_fill[s] = f;
+    }
+    if (*abort_flag && lane == 0) {
+      // Consumers gave up: let copies already in flight land before the CTA exits.
+      int never = 0;
+      for (int s = 0; s < kStages; ++s)
+        if (last_fill[s] >= 0) mbar_wait(full_bar(s), last_fill[s] & 1, &never, 100000000ull);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int gi = lane / LPT;
+  const int j = lane - gi * LPT;
+  float qf[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh) {
+    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D) + j);
+    unpack8(w, qf[hh]);
+  }
+  const float c = p.scale_log2;
+  float m_own = -INFINITY, l_own = 0.f;
+  float acc[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+
+  bool ok = true;
+  for (int it = 0; it < niters; ++it) {
+    const int s = it % kStages;
+    ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / kStages) & 1, abort_flag));
+    if (!ok) break;
+    const int nv = min(kStageTokens, t1 - (t0 + it * kStageTokens));
+    const uint32_t sk = sbase + L::kK + s * L::kStageBytes;
+    const uint32_t sv = sbase + L::kV + s * L::kStageBytes;
+    for (int u = warp; u < UNITS; u += kConsumerWarps) {
+      const int tb = u * TPW + gi * TOK;  // first token of this lane group in the stage
+      float vals[LPT];
+#pragma unroll
+      for (int tt = 0; tt < TOK; ++tt) {
+        float kf[8];
+        unpack8(lds128(sk + (uint32_t)(tb + tt) * L::kRow + 16u * j), kf);
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          float d0 = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) d0 = fmaf(qf[hh][e], kf[e], d0);
+          vals[tt * G + hh] = d0;
+        }
+      }
+      const float score = reduce_scatter<LPT>(vals, j);
+      const bool valid = tb + j / G < nv;
+      const float x = valid ? score * c : -INFINITY;
+      float mx = x;
+#pragma unroll
+      for (int o = G; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_new = fmaxf(m_own, mx);
+      const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_own - m_new);
+      const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+      const float pr = fast_exp2(x - mu);
+      l_own = l_own * alpha + pr;
+      m_own = m_new;
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float ah = __shfl_sync(0xffffffffu, alpha, hh);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[hh][e] *= ah;
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < TOK; ++tt) {
+        float vf[8];
+        unpack8(lds128(sv + (uint32_t)(tb + tt) * L::kRow + 16u * j), vf);
+        const bool tv = tb + tt < nv;
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) {
+          const float ph = __shfl_sync(0xffffffffu, pr, gi * LPT + tt * G + hh);
+          if (tv) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(ph, vf[e], acc[hh][e]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(s));
+  }
+
+  // Merge lane groups of this warp: per head, acc summed over groups, l over all lanes.
+#pragma unroll
+  for (int o = LPT; o < 32; o <<= 1)
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[hh][e] += __shfl_xor_sync(0xffffffffu, acc[hh][e], o);
+  float l_sum = l_own;
+#pragma unroll
+  for (int o = G; o < 32; o <<= 1) l_sum += __shfl_xor_sync(0xffffffffu, l_sum, o);
+
+  // Merge the consumer warps through shared memory (the ring is idle now).
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  float* m_s = reinterpret_cast<float*>(smem);                 // [warps][G]
+  float* l_s = m_s + kConsumerWarps * G;                       // [warps][G]
+  float* a_s = l_s + kConsumerWarps * G;                       // [warps][G][D]
+  if (ok) {
+    if (lane < G) {
+      m_s[warp * G + lane] = m_own;  // lane hh holds head hh
+      l_s[warp * G + lane] = l_sum;
+    }
+    if (gi == 0) {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a_s[(warp * G + hh) * D + 8 * j + e] = acc[hh][e];
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  if (!ok) return;
+  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+    const int hh = idx / D, d = idx - hh * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, m_s[w * G + hh]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kConsumerWarps; ++w) {
+        const float sc = fast_exp2(m_s[w * G + hh] - M);
+        Lsum += l_s[w * G + hh] * sc;
+        O += a_s[(w * G + hh) * D + d] * sc;
+      }
+    }
+    const size_t slot = ((size_t)b * p.Hq + h0 + hh) * p.max_splits + split;
+    p.ws_o[slot * D + d] = Lsum > 0.f ? O / Lsum : 0.f;
+    if (d == 0) p.ws_lse[slot] = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+  }
+}
+
+// One CTA per (sequence, query head): merge the split partials.
+template <int D>
+__global__ void __launch_bounds__(D) decode_combine_kernel(const Params p) {
+  const int bh = blockIdx.x;
+  const int b = bh / p.Hq;
+  const int d = threadIdx.x;
+  const int len = checked_len(p, b, false);
+  const int ns = (len + p.chunk - 1) / p.chunk;
+  const float* lse_s = p.ws_lse + (size_t)bh * p.max_splits;
+  const float* o_s = p.ws_o + (size_t)bh * p.max_splits * D;
+  float M = -INFINITY;
+  for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
+  float out = 0.f, lse = -INFINITY;
+  if (M != -INFINITY) {
+    float Lsum = 0.f;
+    for (int s = 0; s < ns; ++s) Lsum += expf(lse_s[s] - M);
+    lse = M + logf(Lsum);
+    for (int s = 0; s < ns; ++s) out = fmaf(expf(lse_s[s] - lse), o_s[(size_t)s * D + d], out);
+  }
+  p.o[(size_t)bh * D + d] = __float2bfloat16_rn(out);
+  if (p.lse != nullptr && d == 0) p.lse[bh] = lse;
+}
+
+}  // namespace dec
+}  // namespace attn

@@ -1,0 +1,175 @@
+/*
+ * exact_attention_137_b200 -- exact grouped-query attention for NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every call takes plain pointers and sizes; tensors are caller-owned,
+ * contiguous, row-major device memory unless stated otherwise.  Kernel-launching
+ * calls enqueue work on `stream` (a cudaStream_t passed as void*; NULL = legacy
+ * default stream), never synchronise, never allocate, and return a status code.
+ * Invalid arguments are rejected on the host before anything is launched.
+ *
+ * What is computed (page titles abbreviated):
+ *   O = softmax(Q K^T * scale) V per query head, with query head h reading K/V head
+ *   h / (Hq / Hkv) -- the repeat-KV-heads convention of the CSDN interview article
+ *   «注意力变体深挖», section 五 (grouped_query_attention), which also fixes the
+ *   [batch, heads, seq, d_head] layout and the precondition Hq % Hkv == 0.
+ *   Hkv == Hq is MHA and Hkv == 1 is MQA (gocoding blog «different attention
+ *   mechanisms», sections 1-3).  The result is exact: the kernels tile Q/K/V through
+ *   on-chip memory with an online softmax and never write the score matrix to HBM
+ *   (CSDN section 6.2; gocoding section 4).
+ *
+ * Conventions the pages leave open (the readings this library implements):
+ *   - causal: key j is visible to query i iff j <= i + Sk - Sq (lower triangle when
+ *     Sq == Sk; bottom-right aligned otherwise);
+ *   - a query row with no visible key gets O = 0 and LSE = -inf;
+ *   - LSE[row] = ln sum_j exp(scale * q . k_j) over visible keys (natural log).
+ */
+#ifndef EXACT_ATTENTION_137_B200_ATTN_H
+#define EXACT_ATTENTION_137_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------ status codes */
+#define ATTN_OK 0
+#define ATTN_ERR_ARG 1         /* null pointer, non-positive or inconsistent size */
+#define ATTN_ERR_HEADS 2       /* Hq % Hkv != 0 (CSDN «注意力变体深挖» §五 assert) */
+#define ATTN_ERR_UNSUPPORTED 3 /* head dim / dtype / shape combination not built */
+#define ATTN_ERR_CUDA 4        /* a CUDA runtime or driver call failed */
+#define ATTN_ERR_DEVICE 5      /* a kernel flagged an error (bad block id, wait timeout) */
+#define ATTN_ERR_WORKSPACE 6   /* workspace missing, misaligned or too small */
+
+/* ------------------------------------------------------------------ element types */
+#define ATTN_BF16 0 /* bfloat16 storage, fp32 accumulation */
+#define ATTN_F32 1  /* float32 storage and arithmetic (prefill only) */
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char* attn_error_string(int status);
+
+/* Version of this ABI; bumps when a signature changes. */
+int attn_abi_version(void);
+
+/* ------------------------------------------------------------------ prefill forward
+ * attn_fwd: causal or non-causal attention forward that also returns the row LSE.
+ *
+ *   q   [B, Hq,  Sq, D]  dtype        read
+ *   k   [B, Hkv, Sk, D]  dtype        read
+ *   v   [B, Hkv, Sk, D]  dtype        read
+ *   o   [B, Hq,  Sq, D]  dtype        written (must not alias q/k/v)
+ *   lse [B, Hq,  Sq]     float32      written; may be NULL
+ *
+ * D must be 64 or 128.  dtype ATTN_BF16 runs the tensor-core kernel (tcgen05 MMAs
+ * with TMEM accumulators, TMA-fed tiles of 128 queries x 128 keys); q, k, v and o
+ * must be 16-byte aligned.  dtype ATTN_F32 runs a CUDA-core kernel with fp32
+ * arithmetic throughout (the 1e-4 accuracy path).  scale multiplies Q K^T (the pages
+ * use 1/sqrt(D)).  Returns ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_HEADS,
+ * ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA (launch failure).  Sizes are validated on
+ * the host; Sq == 0 or Sk == 0 is allowed (Sk == 0 writes O = 0, LSE = -inf).  q and o
+ * may be NULL only when Sq == 0, k and v only when Sk == 0.  O is normalised by the
+ * row sum of the bf16-rounded probabilities that multiply V (so the weights sum to
+ * one exactly); LSE uses the unrounded fp32 row sum.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
+             int dtype, void* stream);
+
+/* ------------------------------------------------------------------ decode
+ * Single-token decode against a KV cache (CSDN «注意力变体深挖» §七: each step
+ * computes only the new token's Q against the cached K/V; gocoding §5: a paged cache
+ * maps each sequence's logical blocks to physical blocks through a page table).
+ *
+ *   q           [B, Hq, D]                         bf16, read
+ *   k_cache     paged:      [num_blocks, Hkv, block_size, D]   bf16, read
+ *               contiguous: [B, Hkv, block_size, D] (block_size = capacity)
+ *   v_cache     same layout as k_cache
+ *   seqlens     [B] int32 on the device: cached tokens per sequence, INCLUDING the
+ *               current token (the caller appends its K/V before the call)
+ *   block_table [B, max_blocks] int32 on the device, or NULL for a contiguous
+ *               cache.  Logical token t of sequence b lives in physical block
+ *               block_table[b*max_blocks + t/block_size], slot t % block_size.
+ *               Entries past ceil(seqlens[b]/block_size) are never read.
+ *   o           [B, Hq, D] bf16, written
+ *   lse         [B, Hq] float32, written; may be NULL
+ *
+ * max_seqlen must be >= every seqlens[b]; it sizes the split plan and the
+ * workspace.  The work is split along the KV length into chunks (attn_decode_plan);
+ * each split writes a partial (O, LSE) into `workspace` and a combine pass merges
+ * them with the same LSE-weighted rule as the pages' two-way online-softmax merge.
+ * workspace must be device memory of at least attn_decode_workspace_bytes(...) bytes,
+ * 256-byte aligned, and zero-filled before its first use; the library keeps a sticky
+ * error word at its start (read and cleared by attn_decode_check).  Device-side
+ * checks: a block id outside [0, num_blocks), a seqlen above max_seqlen or above
+ * max_blocks*block_size sets that word; the offending tokens are skipped (never
+ * read) and the outputs of that sequence are unspecified.  D must be 64 or 128,
+ * dtype ATTN_BF16, and every row start 16-byte aligned.
+ * Returns ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_HEADS, ATTN_ERR_UNSUPPORTED,
+ * ATTN_ERR_WORKSPACE or ATTN_ERR_CUDA.
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                const int* seqlens, const int* block_table,
+                int block_size, int max_blocks, int num_blocks, int max_seqlen,
+                int B, int Hq, int Hkv, int D, float scale,
+                void* workspace, size_t workspace_bytes,
+                void* o, float* lse, int dtype, void* stream);
+
+/* Bytes of workspace attn_decode needs for these sizes (0 on invalid arguments). */
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen);
+
+/* Split-KV plan (pure host function, no device access):
+ *   G          = largest of 8, 4, 2, 1 dividing g = Hq/Hkv (query heads per CTA);
+ *   streams    = B * Hkv * (g / G);
+ *   splits     = clamp(ceil(2368 / streams), 1, max(1, ceil(max_seqlen / 256)));
+ *   chunk      = max(64, 64 * ceil(ceil(max(max_seqlen,1) / splits) / 64)) tokens;
+ *   max_splits = max(1, ceil(max_seqlen / chunk)).
+ * Sequence b uses ceil(seqlens[b] / chunk) splits (0 when empty).  Any output pointer
+ * may be NULL.  Returns ATTN_OK, ATTN_ERR_ARG or ATTN_ERR_HEADS. */
+int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen,
+                     int* chunk_tokens, int* max_splits, int* heads_per_cta);
+
+/* Synchronises `stream`, reads the sticky error word in `workspace`, clears it, and
+ * returns ATTN_ERR_DEVICE if a decode call since the last check flagged an error
+ * (ATTN_OK otherwise; ATTN_ERR_CUDA if the copy failed). */
+int attn_decode_check(void* workspace, void* stream);
+
+/* ------------------------------------------------------------------ device status
+ * Synchronises `stream` and returns the library-wide device status word of the
+ * current device: 0, or a bitmask of ATTN_DEV_* flags raised by any kernel (for
+ * example a bounded wait that gave up).  clear != 0 resets it.  Returns -1 if the
+ * read failed. */
+#define ATTN_DEV_WAIT_TIMEOUT 1u
+#define ATTN_DEV_BAD_BLOCK 2u
+#define ATTN_DEV_BAD_SEQLEN 4u
+int attn_device_status(int clear, void* stream);
+
+/* Test hook for the bounded waits: launches one CTA that waits on an mbarrier that
+ * nothing completes, giving up after `timeout_ns` nanoseconds (capped at 1e9).  The
+ * kernel then raises ATTN_DEV_WAIT_TIMEOUT in the device status and returns; it
+ * never traps.  Returns the launch status. */
+int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+/* ------------------------------------------------------------------ KV-cache sizing
+ * Bytes of a dense K+V cache: 2 * layers * kv_heads * head_dim * tokens * batch *
+ * elem_bytes (kongchang course summary, "MHA、GQA与MQA": 2 x L x H_kv x d_head x b x
+ * bytes; CSDN «注意力变体深挖» §七 adds the layer factor).  Returns 0 on a negative
+ * argument or on overflow of size_t. */
+size_t attn_kv_cache_bytes(int layers, int kv_heads, int head_dim, long long tokens,
+                           int batch, int elem_bytes);
+
+/* Physical blocks a paged pool needs: sum over b of ceil(seqlens_host[b] /
+ * block_size) (gocoding §5: fixed-size blocks allocated on demand).  seqlens_host is
+ * HOST memory.  Returns -1 on invalid arguments. */
+long long attn_paged_pool_blocks(const int* seqlens_host, int B, int block_size);
+
+/* Bytes of one paged pool (K or V) with num_blocks blocks:
+ * num_blocks * kv_heads * block_size * head_dim * elem_bytes (0 on bad input). */
+size_t attn_paged_pool_bytes(long long num_blocks, int kv_heads, int block_size, int head_dim,
+                             int elem_bytes);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTENTION_137_B200_ATTN_H */

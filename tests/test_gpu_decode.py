@@ -1,0 +1,143 @@
+"""Decode parity: split-KV decode through the C ABI against the fp64 oracle.
+
+Covers contiguous and paged caches, ragged lengths (1 token, page tails, lengths not
+a multiple of the split chunk), odd page sizes, unused NaN-filled pool blocks, MHA /
+GQA / MQA head sharing, D=64 and 128, empty sequences, the device-side block-id check,
+and the two full-size workloads on every output.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import decode_ref
+from exact_attention_137_b200 import _lib, attn_decode, decode_check, decode_workspace, device_status
+from exact_attention_137_b200.workloads import decode_contiguous_inputs, decode_paged_inputs, to_f64
+
+from parity import BF16_TOL, compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+def _run(x, ws=None):
+    g = _gpu(x)
+    o, lse = attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=g["max_seqlen"],
+                         block_table=g["block_table"], block_size=g["block_size"], workspace=ws)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def _ref(x):
+    bt = None if x["block_table"] is None else x["block_table"].numpy()
+    return decode_ref(to_f64(x["q"]), x["k_cache"].float().numpy(), x["v_cache"].float().numpy(),
+                      x["seqlens"].numpy(), block_table=bt, block_size=x["block_size"])
+
+
+@pytest.mark.parametrize("shape", [
+    # B, Hq, Hkv, D, cap, lens
+    (3, 8, 2, 128, 300, [1, 100, 300]),
+    (4, 32, 8, 128, 1100, [1024, 33, 64, 1099]),
+    (2, 4, 4, 64, 200, [200, 17]),        # MHA (one head per CTA)
+    (2, 32, 1, 128, 700, [700, 129]),     # MQA (8 heads per CTA, 4 subgroups)
+    (2, 6, 2, 128, 90, [90, 45]),         # g = 3
+])
+def test_contiguous_small(cuda_lib, shape):
+    B, Hq, Hkv, D, cap, lens = shape
+    x = decode_contiguous_inputs(B, Hq, Hkv, D, cap, 0, 0, seed=sum(lens), seqlens=lens)
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, f"contiguous {shape}")
+
+
+@pytest.mark.parametrize("shape", [
+    # B, Hq, Hkv, D, block_size, lens, extra NaN blocks
+    (3, 8, 2, 128, 16, [1, 100, 513], 5),
+    (4, 32, 8, 128, 16, [512, 8192, 77, 3000], 0),
+    (2, 16, 4, 64, 5, [23, 101], 3),      # page size that does not divide a stage
+    (2, 8, 8, 128, 64, [64, 650], 2),
+    (2, 8, 2, 128, 1, [40, 3], 0),        # one token per page
+])
+def test_paged_small(cuda_lib, shape):
+    B, Hq, Hkv, D, bs, lens, extra = shape
+    x = decode_paged_inputs(B, Hq, Hkv, D, bs, 0, max(lens), seed=bs + B, seqlens=lens, extra_blocks=extra)
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, f"paged {shape}")
+
+
+def test_empty_sequence_gives_zero_and_neg_inf(cuda_lib):
+    x = decode_paged_inputs(3, 8, 2, 128, 16, 0, 50, seed=1, seqlens=[0, 50, 0])
+    o, lse = _run(x)
+    assert torch.all(o[0] == 0) and torch.all(o[2] == 0)
+    assert torch.all(torch.isneginf(lse[0])) and torch.all(torch.isneginf(lse[2]))
+    compare(o, lse, *_ref(x), BF16_TOL, "empty")
+
+
+def test_shared_prefix_blocks(cuda_lib):
+    # Two sequences whose page tables point at the same physical blocks read the same K/V.
+    x = decode_paged_inputs(2, 8, 2, 128, 16, 0, 64, seed=2, seqlens=[64, 64])
+    x["block_table"][1] = x["block_table"][0]
+    x["q"][1] = x["q"][0]
+    o, lse = _run(x)
+    assert torch.equal(o[0], o[1]) and torch.equal(lse[0], lse[1])
+    compare(o, lse, *_ref(x), BF16_TOL, "shared prefix")
+
+
+def test_bad_block_id_is_flagged_not_read(cuda_lib):
+    x = decode_paged_inputs(2, 8, 2, 128, 16, 0, 100, seed=3, seqlens=[100, 40])
+    x["block_table"][1, 1] = x["num_blocks"] + 7  # out of range
+    g = _gpu(x)
+    ws = decode_workspace(2, 8, 2, 128, 100, "cuda")
+    assert device_status(clear=True) == 0
+    attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=100, block_table=g["block_table"],
+                workspace=ws)
+    assert decode_check(ws) == _lib.ATTN_ERR_DEVICE
+    assert decode_check(ws) == _lib.ATTN_OK  # the check clears the sticky word
+    assert device_status(clear=True) & _lib.ATTN_DEV_BAD_BLOCK
+
+
+def test_seqlen_above_max_is_flagged(cuda_lib):
+    x = decode_contiguous_inputs(2, 8, 2, 128, 128, 0, 0, seed=4, seqlens=[128, 100])
+    g = _gpu(x)
+    ws = decode_workspace(2, 8, 2, 128, 64, "cuda")
+    attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=64, workspace=ws)
+    assert decode_check(ws) == _lib.ATTN_ERR_DEVICE
+    assert device_status(clear=True) & _lib.ATTN_DEV_BAD_SEQLEN
+
+
+def test_workspace_reuse_two_calls(cuda_lib):
+    x = decode_paged_inputs(4, 32, 8, 128, 16, 100, 900, seed=6)
+    ws = decode_workspace(4, 32, 8, 128, x["max_seqlen"], "cuda")
+    o1, l1 = _run(x, ws)
+    o2, l2 = _run(x, ws)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert decode_check(ws) == _lib.ATTN_OK
+
+
+def test_full_size_contiguous(cuda_lib):
+    # B=16, Hq=32, Hkv=8, D=128, capacity 4096, lengths U[1024, 4096]: every output.
+    x = decode_contiguous_inputs(16, 32, 8, 128, 4096, 1024, 4096, seed=0)
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, "contiguous B=16")
+
+
+def test_full_size_paged(cuda_lib):
+    # B=64, Hq=32, Hkv=8, D=128, block 16, lengths U[512, 8192], permuted pool: every output.
+    x = decode_paged_inputs(64, 32, 8, 128, 16, 512, 8192, seed=0)
+    assert x["block_table"].shape == (64, 512)
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, "paged B=64")
+
+
+def test_bounded_wait_reports_timeout(cuda_lib):
+    assert device_status(clear=True) == 0
+    assert _lib.selftest_wait_timeout(2_000_000) == 0
+    st = device_status(clear=True)
+    assert st & _lib.ATTN_DEV_WAIT_TIMEOUT
+    assert device_status() == 0
+    # the context is still usable afterwards
+    x = decode_contiguous_inputs(1, 4, 1, 64, 32, 0, 0, seed=7, seqlens=[32])
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, "after timeout")

@@ -1,0 +1,136 @@
+"""Prefill parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Small shapes span several 128-row tiles, ragged tails, every head-grouping path of
+the tensor-core kernel (head pairs, odd leftover head, MHA, MQA), Sq != Sk causal
+alignment and fully masked rows; they are compared on every element.  The full-size
+workloads (S=2048 head-sharing sweep, S=16384 long context with spiked keys) run in
+the launch configuration the bench times and are compared on sampled rows, each
+row exact over its whole visible key range.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention_ref, attention_rows_ref
+from exact_attention_137_b200 import attn_fwd, device_status
+from exact_attention_137_b200.workloads import prefill_inputs, to_f64
+
+from parity import BF16_TOL, F32_TOL, compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, causal, scale=None):
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = attn_fwd(q, k, v, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def _ref(x, causal, scale=None, rows=None):
+    return attention_rows_ref(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), causal=causal, scale=scale,
+                              rows=rows)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_fp32_config(cuda_lib, causal):
+    # B=1, Hq=4, Hkv=2, Sq=Sk=128, D=64, fp32, seed 0, scale 1/sqrt(64).
+    x = prefill_inputs(1, 4, 2, 128, 128, 64, dtype="f32", seed=0)
+    o, lse = _run(x, causal)
+    o_ref, l_ref = _ref(x, causal)
+    compare(o, lse, o_ref, l_ref, F32_TOL, "fp32 tiny")
+
+
+@pytest.mark.parametrize("shape", [(1, 4, 1, 70, 90, 128, True), (2, 2, 2, 33, 300, 64, False),
+                                   (1, 3, 1, 200, 150, 128, True)])
+def test_fp32_ragged(cuda_lib, shape):
+    B, Hq, Hkv, Sq, Sk, D, causal = shape
+    x = prefill_inputs(B, Hq, Hkv, Sq, Sk, D, dtype="f32", seed=3)
+    o, lse = _run(x, causal)
+    compare(o, lse, *_ref(x, causal), F32_TOL, f"fp32 {shape}")
+
+
+BF16_SHAPES = [
+    # B, Hq, Hkv, Sq, Sk, D, causal
+    (1, 4, 2, 128, 128, 64, False),
+    (1, 4, 2, 128, 128, 64, True),
+    (1, 4, 2, 300, 300, 128, False),
+    (1, 4, 2, 300, 300, 128, True),
+    (2, 8, 1, 257, 257, 64, True),     # MQA, ragged tail
+    (1, 3, 3, 520, 520, 128, True),    # MHA: odd groups, pairs of query tiles
+    (1, 6, 2, 384, 384, 128, True),    # g = 3: a head pair plus a leftover head
+    (1, 4, 2, 100, 300, 128, True),    # Sq < Sk: bottom-right aligned mask
+    (1, 4, 2, 300, 100, 128, True),    # Sq > Sk: fully masked leading rows
+    (1, 2, 1, 130, 129, 128, False),
+    (1, 2, 1, 1, 1, 128, True),
+    (1, 2, 2, 5, 7, 64, False),
+    (3, 4, 4, 256, 640, 64, False),
+]
+
+
+@pytest.mark.parametrize("shape", BF16_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_small_all_elements(cuda_lib, shape):
+    B, Hq, Hkv, Sq, Sk, D, causal = shape
+    x = prefill_inputs(B, Hq, Hkv, Sq, Sk, D, dtype="bf16", seed=sum(shape))
+    o, lse = _run(x, causal)
+    compare(o, lse, *_ref(x, causal), BF16_TOL, f"bf16 {shape}")
+
+
+def test_bf16_empty_keys(cuda_lib):
+    x = prefill_inputs(1, 2, 1, 9, 0, 64, dtype="bf16", seed=1)
+    o, lse = _run(x, False)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_bf16_large_scores_and_scale(cuda_lib):
+    # Scores of several hundred (scale 1): the online max must keep exp in range.
+    x = prefill_inputs(1, 4, 2, 256, 256, 128, dtype="bf16", seed=9)
+    x["q"] = (x["q"].float() * 4).to(torch.bfloat16)
+    o, lse = _run(x, True, scale=1.0)
+    compare(o, lse, *_ref(x, True, scale=1.0), BF16_TOL, "large scores")
+
+
+def test_bf16_decode_row_equals_last_causal_row(cuda_lib):
+    from exact_attention_137_b200 import attn_decode
+
+    x = prefill_inputs(2, 8, 2, 200, 200, 128, dtype="bf16", seed=5)
+    o, lse = _run(x, True)
+    q = x["q"][:, :, -1].contiguous().cuda()
+    seqlens = torch.full((2,), 200, dtype=torch.int32, device="cuda")
+    od, ld = attn_decode(q, x["k"].cuda(), x["v"].cuda(), seqlens, max_seqlen=200)
+    torch.cuda.synchronize()
+    assert (od.float() - o[:, :, -1].float()).abs().max().item() <= 2e-2
+    assert (ld - lse[:, :, -1]).abs().max().item() <= 1e-3
+
+
+def _sample_rows(S, n, seed, must=()):
+    rows = set(range(min(8, S))) | set(range(max(0, S - 8), S)) | {int(r) for r in must if r < S}
+    rng = np.random.Generator(np.random.PCG64(seed))
+    while len(rows) < min(n, S):
+        rows.add(int(rng.integers(0, S)))
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("hkv", [32, 8, 1])
+def test_full_size_head_sharing_sweep_sampled(cuda_lib, hkv):
+    # B=2, Hq=32, Hkv in {32, 8, 1}, Sq=Sk=2048, D=128, bf16, causal (the bench's workload).
+    x = prefill_inputs(2, 32, hkv, 2048, 2048, 128, dtype="bf16", seed=0)
+    o, lse = _run(x, True)
+    rows = _sample_rows(2048, 192, seed=hkv)
+    o_ref, l_ref = _ref(x, True, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, l_ref, BF16_TOL, f"S=2048 Hkv={hkv}")
+
+
+def test_full_size_long_context_spiked_sampled(cuda_lib):
+    # B=1, Hq=64, Hkv=8, S=16384, D=128, bf16, causal, 0.1% of key rows x8.
+    x = prefill_inputs(1, 64, 8, 16384, 16384, 128, dtype="bf16", seed=0, spike_frac=0.001)
+    o, lse = _run(x, True)
+    spikes = x["spike_rows"].reshape(-1)
+    rows = _sample_rows(16384, 192, seed=4, must=spikes[:: max(1, spikes.size // 64)])
+    o_ref, l_ref = _ref(x, True, rows=rows)
+    compare(o[:, :, rows], lse[:, :, rows], o_ref, l_ref, BF16_TOL, "S=16384 spiked")
+
+
+def test_no_device_error_raised(cuda_lib):
+    assert device_status(clear=True) == 0

@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The shared library loads on a CPU-only machine (the CUDA runtime is linked in
+statically); these tests call only functions that validate arguments or do host
+arithmetic, never a kernel.
+"""
+
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from exact_attention_137_b200 import _lib
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_137_b200 import build
+
+    build.build()
+    return _lib.load()
+
+
+def test_exports_every_declared_function(lib):
+    names = _lib.header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/attn.h but not exported"
+    assert lib.attn_abi_version() == 1
+
+
+def test_error_strings(lib):
+    for code in range(0, 7):
+        assert _lib.error_string(code)
+    assert _lib.error_string(99) == "unknown status"
+
+
+def test_kv_cache_bytes_match_pages_and_oracle(lib):
+    with open(os.path.join(GOLDEN, "kv_cache_sizes.txt"), encoding="utf-8") as f:
+        for line in f:
+            if not line.strip() or line.startswith("#"):
+                continue
+            vals = [int(x) for x in line.split("|")[0].split()]
+            assert _lib.kv_cache_bytes(*vals[:6]) == vals[6]
+    rng = np.random.Generator(np.random.PCG64(0))
+    for _ in range(200):
+        a = [int(x) for x in rng.integers(0, 100, size=6)]
+        assert _lib.kv_cache_bytes(*a) == oracle.kv_cache_bytes_ref(*a)
+    assert _lib.kv_cache_bytes(-1, 1, 1, 1, 1, 1) == 0
+
+
+def test_paged_pool_blocks_match_oracle(lib):
+    rng = np.random.Generator(np.random.PCG64(1))
+    for bs in (1, 5, 16, 64):
+        lens = rng.integers(0, 9000, size=64)
+        assert _lib.paged_pool_blocks(lens.tolist(), bs) == oracle.paged_pool_blocks_ref(lens, bs)
+    assert _lib.paged_pool_blocks([3], 0) == -1
+    assert _lib.paged_pool_blocks([-3], 4) == -1
+    assert _lib.paged_pool_bytes(10, 8, 16, 128, 2) == 10 * 8 * 16 * 128 * 2
+
+
+def test_decode_plan_bit_exact_vs_restatement(lib):
+    rng = np.random.Generator(np.random.PCG64(2))
+    cases = [(16, 32, 8, 4096), (64, 32, 8, 8192), (1, 1, 1, 0), (1, 4, 4, 1), (3, 32, 1, 100000),
+             (2, 6, 2, 77), (7, 12, 4, 65536)]
+    for _ in range(300):
+        hkv = int(rng.choice([1, 2, 4, 8, 16]))
+        g = int(rng.choice([1, 2, 3, 4, 5, 6, 8, 16, 32]))
+        cases.append((int(rng.integers(1, 300)), hkv * g, hkv, int(rng.integers(0, 200000))))
+    for B, hq, hkv, L in cases:
+        assert _lib.decode_plan(B, hq, hkv, L) == oracle.decode_plan_ref(B, hq, hkv, L), (B, hq, hkv, L)
+
+
+def test_decode_workspace_bytes_formula(lib):
+    for B, hq, hkv, d, L in [(16, 32, 8, 128, 4096), (64, 32, 8, 128, 8192), (1, 4, 1, 64, 10)]:
+        chunk, ms, _ = oracle.decode_plan_ref(B, hq, hkv, L)
+        lse_bytes = -(-(B * hq * ms * 4) // 256) * 256
+        assert _lib.decode_workspace_bytes(B, hq, hkv, d, L) == 256 + lse_bytes + B * hq * ms * d * 4
+    assert _lib.decode_workspace_bytes(0, 1, 1, 64, 1) == 0
+
+
+FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails validation first
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(q=None), _lib.ATTN_ERR_ARG),
+    (dict(k=None), _lib.ATTN_ERR_ARG),
+    (dict(B=0), _lib.ATTN_ERR_ARG),
+    (dict(Hkv=3), _lib.ATTN_ERR_HEADS),
+    (dict(D=96), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=7), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), _lib.ATTN_ERR_ARG),
+    (dict(q=ctypes.c_void_p((1 << 20) + 8)), _lib.ATTN_ERR_ARG),  # bf16 path needs 16-byte alignment
+])
+def test_fwd_rejects_bad_arguments_before_launch(lib, args, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=4, Hkv=2, Sq=8, Sk=8, D=64, scale=0.125,
+             causal=0, dtype=_lib.ATTN_BF16, stream=None)
+    a.update(args)
+    st = lib.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Sk"],
+                      a["D"], a["scale"], a["causal"], a["dtype"], a["stream"])
+    assert st == code
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(seqlens=None), _lib.ATTN_ERR_ARG),
+    (dict(Hkv=3), _lib.ATTN_ERR_HEADS),
+    (dict(D=80), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(dtype=_lib.ATTN_F32), _lib.ATTN_ERR_UNSUPPORTED),
+    (dict(ws=None), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws_bytes=16), _lib.ATTN_ERR_WORKSPACE),
+    (dict(ws=ctypes.c_void_p((1 << 20) + 16)), _lib.ATTN_ERR_WORKSPACE),
+    (dict(max_blocks=0), _lib.ATTN_ERR_ARG),
+    (dict(block_size=0), _lib.ATTN_ERR_ARG),
+])
+def test_decode_rejects_bad_arguments_before_launch(lib, args, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, seqlens=FAKE, table=FAKE, block_size=16, max_blocks=4, num_blocks=8,
+             max_seqlen=64, B=2, Hq=4, Hkv=2, D=128, scale=0.1, ws=FAKE, ws_bytes=1 << 30, o=FAKE, lse=None,
+             dtype=_lib.ATTN_BF16, stream=None)
+    a.update(args)
+    st = lib.attn_decode(a["q"], a["k"], a["v"], a["seqlens"], a["table"], a["block_size"], a["max_blocks"],
+                         a["num_blocks"], a["max_seqlen"], a["B"], a["Hq"], a["Hkv"], a["D"], a["scale"], a["ws"],
+                         a["ws_bytes"], a["o"], a["lse"], a["dtype"], a["stream"])
+    assert st == code
