@@ -272,7 +272,7 @@ def run_ours(args, rank, world, local):
 
     calls = [("prefill_hkv%d" % c["hkv"], (lambda c=c: run_prefill(c))) for c in pre]
     calls += [("decode_paged", lambda: run_decode(paged)), ("decode_contiguous", lambda: run_decode(contig))]
-    launches_per_step = len(pre) * 1 + 2 * 2
+    launches_per_step = len(pre) + 2  # one prefill kernel per call, one decode kernel per call
     nev = len(calls)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nev)]
           for _ in range(args.steps)]
@@ -355,7 +355,7 @@ def run_ours(args, rank, world, local):
         ms = max_over_ranks(per_call[name], world)
         gbs = g["bytes"] / (ms * 1e-3) / 1e9
         return {"workload": spec_name, "ms": ms, "GB/s": gbs, "kv_bytes": g["kv_bytes"], "bytes": g["bytes"],
-                "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "kernels": ["split", "combine"]}
+                "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "kernels": ["decode_split_kernel (split partials + merge by the last split)"]}
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

@@ -48,6 +48,7 @@ _SIGS = {
     "attn_decode_check": (_c_int, [_vp, _vp]),
     "attn_device_status": (_c_int, [_c_int, _vp]),
     "attn_selftest_wait_timeout": (_c_int, [_ull, _vp]),
+    "attn_selftest_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
     "attn_kv_cache_bytes": (_size_t, [_c_int, _c_int, _c_int, _ll, _c_int, _c_int]),
     "attn_paged_pool_blocks": (_ll, [_ip, _c_int, _c_int]),
     "attn_paged_pool_bytes": (_size_t, [_ll, _c_int, _c_int, _c_int, _c_int]),
@@ -227,6 +228,16 @@ def device_status(clear: bool = False, stream=None) -> int:
 
 def selftest_wait_timeout(timeout_ns: int, stream=None) -> int:
     return int(load().attn_selftest_wait_timeout(int(timeout_ns), ctypes.c_void_p(_stream_ptr(stream))))
+
+
+def selftest_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """2^x by the polynomial the prefill kernel uses for part of its exponentials."""
+    if x.dtype != torch.float32 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    _check(load().attn_selftest_exp2_poly(_ptr(x), _ptr(y), x.numel(), ctypes.c_void_p(_stream_ptr(stream))),
+           "attn_selftest_exp2_poly")
+    return y
 
 
 # ------------------------------------------------------------------ KV-cache sizing (host only)

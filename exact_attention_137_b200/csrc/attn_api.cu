@@ -145,7 +145,7 @@ bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
   const long long streams = (long long)B * Hkv * (g / G);
   long long splits = cdiv(kDecodeTargetCtas, streams);
   const long long cap = std::max(1LL, cdiv(max_seqlen, 256));
-  splits = std::max(1LL, std::min(splits, cap));
+  splits = std::max(1LL, std::min(std::min(splits, cap), (long long)attn::dec::kMaxSplits));
   const long long per = cdiv(std::max(max_seqlen, 1), splits);
   const long long chunk = std::max(64LL, 64 * cdiv(per, 64));
   out->chunk = (int)chunk;
@@ -154,9 +154,22 @@ bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
   return true;
 }
 
-size_t ws_lse_bytes(int B, int Hq, int ms) {
-  size_t n = (size_t)B * Hq * ms * sizeof(float);
-  return (n + 255) & ~size_t(255);
+inline size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Workspace layout: [error word | 256 B] [split counters, B*Hkv*(g/G) int32, 256-aligned]
+// [partial LSE, B*Hq*max_splits fp32, 256-aligned] [partial O, B*Hq*max_splits*D fp32].
+struct WsLayout {
+  size_t cnt, lse, o, total;
+};
+
+WsLayout ws_layout(int B, int Hq, int Hkv, int D, const DecodePlan& pl) {
+  WsLayout w;
+  const size_t streams = (size_t)B * Hkv * ((Hq / Hkv) / pl.G);
+  w.cnt = kWsHeader;
+  w.lse = w.cnt + round256(streams * sizeof(int));
+  w.o = w.lse + round256((size_t)B * Hq * pl.max_splits * sizeof(float));
+  w.total = w.o + (size_t)B * Hq * pl.max_splits * D * sizeof(float);
+  return w;
 }
 
 template <int D, int G>
@@ -178,8 +191,6 @@ int launch_decode_split(const attn::dec::Params& p, cudaStream_t st) {
   }
   dim3 grid((unsigned)p.max_splits, (unsigned)(p.Hkv * p.nsub), (unsigned)p.B);
   kern<<<grid, attn::dec::kThreads, Lay::kBytes, st>>>(p);
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
-  attn::dec::decode_combine_kernel<D><<<(unsigned)(p.B * p.Hq), D, 0, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -208,6 +219,16 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   attn::mbar_wait(b, 0, &abort_flag, limit_ns);
 }
 
+__global__ void selftest_exp2_kernel(const float* x, float* y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i >= n) return;
+  const float x0 = x[i], x1 = i + 1 < n ? x[i + 1] : 0.f;
+  float y0, y1;
+  attn::f2unpack(attn::exp2_poly2(attn::f2pack(x0, x1)), y0, y1);
+  y[i] = y0;
+  if (i + 1 < n) y[i + 1] = y1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -229,7 +250,8 @@ int attn_abi_version(void) { return kAbiVersion; }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
              int Sk, int D, float scale, int causal, int dtype, void* stream) {
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || !std::isfinite(scale)) return ATTN_ERR_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || !std::isfinite(scale) || !(scale > 0.f))
+    return ATTN_ERR_ARG;
   // q/o may be NULL only when Sq == 0, k/v only when Sk == 0 (nothing is read or written).
   if ((Sq > 0 && (!q || !o)) || (Sk > 0 && (!k || !v))) return ATTN_ERR_ARG;
   if (Hq % Hkv) return ATTN_ERR_HEADS;
@@ -270,7 +292,7 @@ int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int* chunk_tokens, 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen) {
   DecodePlan pl;
   if (D <= 0 || !decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return 0;
-  return kWsHeader + ws_lse_bytes(B, Hq, pl.max_splits) + (size_t)B * Hq * pl.max_splits * D * sizeof(float);
+  return ws_layout(B, Hq, Hkv, D, pl).total;
 }
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
@@ -314,9 +336,11 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.max_splits = pl.max_splits;
   p.nsub = (Hq / Hkv) / pl.G;
   p.scale_log2 = scale * attn::kLog2e;
+  const WsLayout wl = ws_layout(B, Hq, Hkv, D, pl);
   p.ws_err = reinterpret_cast<unsigned int*>(ws);
-  p.ws_lse = reinterpret_cast<float*>(ws + kWsHeader);
-  p.ws_o = reinterpret_cast<float*>(ws + kWsHeader + ws_lse_bytes(B, Hq, pl.max_splits));
+  p.ws_cnt = reinterpret_cast<int*>(ws + wl.cnt);
+  p.ws_lse = reinterpret_cast<float*>(ws + wl.lse);
+  p.ws_o = reinterpret_cast<float*>(ws + wl.o);
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   cudaStream_t st = as_stream(stream);
@@ -353,6 +377,14 @@ int attn_device_status(int clear, void* stream) {
 int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream) {
   if (timeout_ns > 1000000000ull) timeout_ns = 1000000000ull;
   selftest_wait_kernel<<<1, 32, 0, as_stream(stream)>>>(timeout_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (!x || !y || n < 0) return ATTN_ERR_ARG;
+  if (n == 0) return ATTN_OK;
+  const int pairs = (n + 1) / 2;
+  selftest_exp2_kernel<<<(pairs + 255) / 256, 256, 0, as_stream(stream)>>>(x, y, n);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

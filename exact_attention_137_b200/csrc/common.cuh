@@ -238,6 +238,63 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Packed fp32 pairs (Blackwell FFMA2/FADD2/FMUL2): two fp32 lanes in one 64-bit register.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^y for a pair of finite y on the FMA pipe (keeps the MUFU free for other elements).
+// Split y = n + f with n = rint(y) (adding and subtracting 1.5 * 2^23) and f in
+// [-1/2, 1/2]; 2^f by the degree-3 polynomial of least maximum relative error on
+// [-1/2, 1/2] (Remez exchange, max relative error 7.5e-5); 2^n is applied by adding n
+// to the exponent field.  y is clamped to >= -126 so the exponent never wraps; results
+// below 2^-126 come out as tiny positive numbers instead of 0, which no sum notices.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t y2) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  float y0, y1;
+  f2unpack(y2, y0, y1);
+  y0 = fmaxf(y0, -126.f);
+  y1 = fmaxf(y1, -126.f);
+  const uint64_t y = f2pack(y0, y1);
+  const uint64_t t = fadd2(y, f2pack(kShift, kShift));
+  const uint64_t n = fadd2(t, f2pack(-kShift, -kShift));
+  const uint64_t f = ffma2(n, f2pack(-1.f, -1.f), y);
+  uint64_t p = ffma2(f2pack(0.0551716685f, 0.0551716685f), f, f2pack(0.2426111251f, 0.2426111251f));
+  p = ffma2(p, f, f2pack(0.6932609677f, 0.6932609677f));
+  p = ffma2(p, f, f2pack(0.9999280572f, 0.9999280572f));
+  float p0, p1, t0, t1;
+  f2unpack(p, p0, p1);
+  f2unpack(t, t0, t1);
+  p0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  p1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+  return f2pack(p0, p1);
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -29,6 +29,7 @@ constexpr int kStageTokens = 32;
 constexpr int kStages = 4;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxSplits = 128;  // the plan never splits a sequence into more chunks
 
 struct Params {
   const __nv_bfloat16* q;
@@ -43,6 +44,7 @@ struct Params {
   float* ws_o;    // [B, Hq, max_splits, D]
   float* ws_lse;  // [B, Hq, max_splits]
   unsigned int* ws_err;
+  int* ws_cnt;    // [B, Hkv * nsub] splits finished; the last one merges and resets it
   __nv_bfloat16* o;
   float* lse;
 };
@@ -131,6 +133,15 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   const int split = blockIdx.x;
   const int len = checked_len(p, b, split == 0 && blockIdx.y == 0 && threadIdx.x == 0);
   const int nsplit = (len + p.chunk - 1) / p.chunk;
+  const int kvh0 = blockIdx.y / p.nsub;
+  const int hbase = kvh0 * (p.Hq / p.Hkv) + (blockIdx.y - kvh0 * p.nsub) * G;
+  if (nsplit == 0 && split == 0) {  // empty sequence: O = 0, LSE = -inf
+    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
+      const int hh = idx / D, d = idx - hh * D;
+      p.o[((size_t)b * p.Hq + hbase + hh) * D + d] = __float2bfloat16_rn(0.f);
+      if (p.lse != nullptr && d == 0) p.lse[(size_t)b * p.Hq + hbase + hh] = -INFINITY;
+    }
+  }
   if (split >= nsplit) return;
   const int t0 = split * p.chunk;
   const int t1 = min(len, t0 + p.chunk);
@@ -216,19 +227,22 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   // -------------------------------------------------------------- consumers
   const int gi = lane / LPT;
   const int j = lane - gi * LPT;
-  float qf[G][8];
+  uint64_t q2[G][4];  // this lane's 8 query elements per head, as fp32 pairs
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
     const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D) + j);
-    unpack8(w, qf[hh]);
+    q2[hh][0] = f2pack(bf16lo(w.x), bf16hi(w.x));
+    q2[hh][1] = f2pack(bf16lo(w.y), bf16hi(w.y));
+    q2[hh][2] = f2pack(bf16lo(w.z), bf16hi(w.z));
+    q2[hh][3] = f2pack(bf16lo(w.w), bf16hi(w.w));
   }
   const float c = p.scale_log2;
   float m_own = -INFINITY, l_own = 0.f;
-  float acc[G][8];
+  uint64_t acc[G][4];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[hh][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[hh][e] = 0ull;
 
   bool ok = true;
   for (int it = 0; it < niters; ++it) {
@@ -243,14 +257,18 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
       float vals[LPT];
 #pragma unroll
       for (int tt = 0; tt < TOK; ++tt) {
-        float kf[8];
-        unpack8(lds128(sk + (uint32_t)(tb + tt) * L::kRow + 16u * j), kf);
+        const uint4 w = lds128(sk + (uint32_t)(tb + tt) * L::kRow + 16u * j);
+        const uint64_t k0 = f2pack(bf16lo(w.x), bf16hi(w.x)), k1 = f2pack(bf16lo(w.y), bf16hi(w.y));
+        const uint64_t k2 = f2pack(bf16lo(w.z), bf16hi(w.z)), k3 = f2pack(bf16lo(w.w), bf16hi(w.w));
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
-          float d0 = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) d0 = fmaf(qf[hh][e], kf[e], d0);
-          vals[tt * G + hh] = d0;
+          uint64_t d2 = fmul2(q2[hh][0], k0);
+          d2 = ffma2(q2[hh][1], k1, d2);
+          d2 = ffma2(q2[hh][2], k2, d2);
+          d2 = ffma2(q2[hh][3], k3, d2);
+          float lo, hi;
+          f2unpack(d2, lo, hi);
+          vals[tt * G + hh] = lo + hi;
         }
       }
       const float score = reduce_scatter<LPT>(vals, j);
@@ -269,21 +287,26 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
           const float ah = __shfl_sync(0xffffffffu, alpha, hh);
+          const uint64_t a2 = f2pack(ah, ah);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[hh][e] *= ah;
+          for (int e = 0; e < 4; ++e) acc[hh][e] = fmul2(acc[hh][e], a2);
         }
       }
 #pragma unroll
       for (int tt = 0; tt < TOK; ++tt) {
-        float vf[8];
-        unpack8(lds128(sv + (uint32_t)(tb + tt) * L::kRow + 16u * j), vf);
+        const uint4 w = lds128(sv + (uint32_t)(tb + tt) * L::kRow + 16u * j);
+        const uint64_t v0 = f2pack(bf16lo(w.x), bf16hi(w.x)), v1 = f2pack(bf16lo(w.y), bf16hi(w.y));
+        const uint64_t v2 = f2pack(bf16lo(w.z), bf16hi(w.z)), v3 = f2pack(bf16lo(w.w), bf16hi(w.w));
         const bool tv = tb + tt < nv;
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) {
           const float ph = __shfl_sync(0xffffffffu, pr, gi * LPT + tt * G + hh);
           if (tv) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[hh][e] = fmaf(ph, vf[e], acc[hh][e]);
+            const uint64_t p2 = f2pack(ph, ph);
+            acc[hh][0] = ffma2(p2, v0, acc[hh][0]);
+            acc[hh][1] = ffma2(p2, v1, acc[hh][1]);
+            acc[hh][2] = ffma2(p2, v2, acc[hh][2]);
+            acc[hh][3] = ffma2(p2, v3, acc[hh][3]);
           }
         }
       }
@@ -293,12 +316,17 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   }
 
   // Merge lane groups of this warp: per head, acc summed over groups, l over all lanes.
+  float accf[G][8];
+#pragma unroll
+  for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f2unpack(acc[hh][e], accf[hh][2 * e], accf[hh][2 * e + 1]);
 #pragma unroll
   for (int o = LPT; o < 32; o <<= 1)
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[hh][e] += __shfl_xor_sync(0xffffffffu, acc[hh][e], o);
+      for (int e = 0; e < 8; ++e) accf[hh][e] += __shfl_xor_sync(0xffffffffu, accf[hh][e], o);
   float l_sum = l_own;
 #pragma unroll
   for (int o = G; o < 32; o <<= 1) l_sum += __shfl_xor_sync(0xffffffffu, l_sum, o);
@@ -308,6 +336,12 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   float* m_s = reinterpret_cast<float*>(smem);                 // [warps][G]
   float* l_s = m_s + kConsumerWarps * G;                       // [warps][G]
   float* a_s = l_s + kConsumerWarps * G;                       // [warps][G][D]
+  // Outside the ring: in-flight copies of an aborted call must not touch these.
+  volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  // Any consumer that gave up set *abort_flag; snapshot it between two barriers so that
+  // every consumer warp takes the same branch below (named barriers never time out).
+  if (threadIdx.x == 0) *ok_s = (*abort_flag == 0);
   if (ok) {
     if (lane < G) {
       m_s[warp * G + lane] = m_own;  // lane hh holds head hh
@@ -317,11 +351,12 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
 #pragma unroll
       for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a_s[(warp * G + hh) * D + 8 * j + e] = acc[hh][e];
+        for (int e = 0; e < 8; ++e) a_s[(warp * G + hh) * D + 8 * j + e] = accf[hh][e];
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  if (!ok) return;
+  if (!*ok_s) return;
+  const size_t bh0 = (size_t)b * p.Hq + h0;
   for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
     const int hh = idx / D, d = idx - hh * D;
     float M = -INFINITY;
@@ -336,33 +371,67 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
         O += a_s[(w * G + hh) * D + d] * sc;
       }
     }
-    const size_t slot = ((size_t)b * p.Hq + h0 + hh) * p.max_splits + split;
-    p.ws_o[slot * D + d] = Lsum > 0.f ? O / Lsum : 0.f;
-    if (d == 0) p.ws_lse[slot] = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+    const float o_val = Lsum > 0.f ? O / Lsum : 0.f;
+    const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+    if (nsplit == 1) {  // the only split: write the result directly
+      p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);
+      if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_val;
+    } else {
+      const size_t slot = (bh0 + hh) * p.max_splits + split;
+      p.ws_o[slot * D + d] = o_val;
+      if (d == 0) p.ws_lse[slot] = lse_val;
+    }
   }
-}
+  if (nsplit == 1) return;
 
-// One CTA per (sequence, query head): merge the split partials.
-template <int D>
-__global__ void __launch_bounds__(D) decode_combine_kernel(const Params p) {
-  const int bh = blockIdx.x;
-  const int b = bh / p.Hq;
-  const int d = threadIdx.x;
-  const int len = checked_len(p, b, false);
-  const int ns = (len + p.chunk - 1) / p.chunk;
-  const float* lse_s = p.ws_lse + (size_t)bh * p.max_splits;
-  const float* o_s = p.ws_o + (size_t)bh * p.max_splits * D;
-  float M = -INFINITY;
-  for (int s = 0; s < ns; ++s) M = fmaxf(M, lse_s[s]);
-  float out = 0.f, lse = -INFINITY;
-  if (M != -INFINITY) {
-    float Lsum = 0.f;
-    for (int s = 0; s < ns; ++s) Lsum += expf(lse_s[s] - M);
-    lse = M + logf(Lsum);
-    for (int s = 0; s < ns; ++s) out = fmaf(expf(lse_s[s] - lse), o_s[(size_t)s * D + d], out);
+  // The last split of this (sequence, head group) to finish merges all partials.
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  int* cnt = p.ws_cnt + (size_t)b * gridDim.y + blockIdx.y;
+  if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == nsplit - 1);
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  if (!*last_s) return;
+  __threadfence();
+  // Stage the partial LSEs in shared memory (one independent load per thread), turn them
+  // into merge weights exp(lse_s - LSE), then combine the partial outputs.
+  float* w_s = reinterpret_cast<float*>(smem);  // [G][max_splits]
+  float* lse_f = w_s + G * kMaxSplits;          // [G]
+  for (int idx = threadIdx.x; idx < G * nsplit; idx += kConsumerWarps * 32) {
+    const int hh = idx / nsplit, sp = idx - hh * nsplit;
+    w_s[hh * kMaxSplits + sp] = __ldcg(p.ws_lse + (bh0 + hh) * p.max_splits + sp);
   }
-  p.o[(size_t)bh * D + d] = __float2bfloat16_rn(out);
-  if (p.lse != nullptr && d == 0) p.lse[bh] = lse;
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  if (threadIdx.x < G) {
+    float* w = w_s + threadIdx.x * kMaxSplits;
+    float M = -INFINITY;
+    for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, w[sp]);
+    float lse = -INFINITY;
+    if (M != -INFINITY) {
+      float Lsum = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) Lsum += expf(w[sp] - M);
+      lse = M + logf(Lsum);
+    }
+    for (int sp = 0; sp < nsplit; ++sp) w[sp] = lse == -INFINITY ? 0.f : expf(w[sp] - lse);
+    lse_f[threadIdx.x] = lse;
+  }
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
+  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+    const int hh = idx / D, d = idx - hh * D;
+    const float* w = w_s + hh * kMaxSplits;
+    const float* o_s = p.ws_o + (bh0 + hh) * p.max_splits * D + d;
+    float out0 = 0.f, out1 = 0.f, out2 = 0.f, out3 = 0.f;
+    int sp = 0;
+    for (; sp + 4 <= nsplit; sp += 4) {
+      out0 = fmaf(w[sp], __ldcg(o_s + (size_t)sp * D), out0);
+      out1 = fmaf(w[sp + 1], __ldcg(o_s + (size_t)(sp + 1) * D), out1);
+      out2 = fmaf(w[sp + 2], __ldcg(o_s + (size_t)(sp + 2) * D), out2);
+      out3 = fmaf(w[sp + 3], __ldcg(o_s + (size_t)(sp + 3) * D), out3);
+    }
+    for (; sp < nsplit; ++sp) out0 = fmaf(w[sp], __ldcg(o_s + (size_t)sp * D), out0);
+    p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
+    if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
+  }
+  if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
 }
 
 }  // namespace dec

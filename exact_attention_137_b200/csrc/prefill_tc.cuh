@@ -12,15 +12,24 @@
 //    tiles of that head.
 //  * warp 0 (one thread) streams Q once and K/V tiles of 128 keys through a 2-stage
 //    shared-memory ring with TMA (128-byte swizzle).
-//  * warp 1 (one thread) issues tcgen05 MMAs: S_i = Q_i K^T (A, B from shared memory)
-//    into TMEM, and O_i += P_i V with P_i read from TMEM (it overwrites S_i as bf16).
-//  * warps 2-5 and 6-9 are the softmax warpgroups of slot 0 and 1.  TMEM lane r holds
+//  * warp 1 (one thread) issues the tcgen05 MMAs: S_i = Q_i K^T (A, B from shared
+//    memory) into TMEM, and O_i += P_i V with P_i read from TMEM (it overwrites S_i as
+//    bf16).  The issue order PV_0, S_0, PV_1, S_1 makes each slot's softmax overlap the
+//    other slot's MMAs (MMAs of one thread run in order, so no completion wait is needed
+//    between PV_i(j) and the S_i(j+1) that overwrites P_i).
+//  * warps 4-7 and 8-11 are the softmax warpgroups of slot 0 and 1.  TMEM lane r holds
 //    query row r, so each thread owns one full row: its row max and row sum need no
-//    cross-lane reduction.  Scores are scaled into the log2 domain with one FFMA and
-//    exponentiated with ex2.  The output is rescaled only when the running max grows
-//    by more than 2^8 (the final O / l uses the same stale reference, so this is exact).
+//    cross-lane reduction.  Scores are scaled into the log2 domain with one packed FFMA
+//    and exponentiated with ex2; P is truncated to bf16 with a byte permute and O is
+//    normalised by the sum of the truncated P.  P is handed to the MMA issuer in two
+//    halves of 64 keys, so the first four PV MMAs run while the second half is still
+//    being exponentiated.
+//  * Reference max: a row's first tile takes the full row max.  Later tiles exponentiate
+//    against the current reference m without a max pass, after checking (max of the
+//    second half, sum of the first half) that no value exceeds 2^64; otherwise the tile
+//    is redone with the max update.  O is rescaled only when the max grows by more than
+//    2^8.  All of this is exact: O and l always share one reference.
 //  * TMEM (512 columns): S_0 | S_1 | O_0 | O_1.
-//  * While one slot runs its softmax the tensor pipe works on the other slot.
 #pragma once
 
 #include <cuda.h>
@@ -32,8 +41,19 @@ namespace tc {
 
 constexpr int BM = 128;  // query rows per tile (MMA M)
 constexpr int BN = 128;  // keys per K/V tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Register split (setmaxnreg): the launch gives every thread 168 registers (65536 / 384
+// rounded down to a multiple of 8), i.e. 64512 in total.  Warpgroup 0 (TMA, MMA, two
+// idle warps) gives registers to the two softmax warpgroups; the split per
+// head dim is the one with the fewest spills (D=128: 64 * 128 + 216 * 256 = 63488;
+// D=64: 56 * 128 + 224 * 256 = 64512).
+template <int D>
+struct Regs {
+  static constexpr int kControl = D == 128 ? 64 : 56;
+  static constexpr int kSoftmax = D == 128 ? 216 : 224;
+};
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kFastBound = 64.0f;        // log2 units: fast-path values stay below 2^64
 
 template <int D>
 struct Layout {
@@ -43,7 +63,7 @@ struct Layout {
   static constexpr int kK = 2 * kTile;      // K[2]
   static constexpr int kV = 4 * kTile;      // V[2]
   static constexpr int kBar = 6 * kTile;
-  static constexpr int kNumBars = 16;
+  static constexpr int kNumBars = 20;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
@@ -54,14 +74,15 @@ struct Layout {
 // barrier indices
 enum : int {
   kBarQ = 0,
-  kBarKFull = 1,   // [2]
-  kBarKEmpty = 3,  // [2]
+  kBarKFull = 1,   // [2] TMA bytes landed
+  kBarKEmpty = 3,  // [2] MMAs that read the stage have completed
   kBarVFull = 5,   // [2]
   kBarVEmpty = 7,  // [2]
   kBarSFull = 9,   // [2] per slot: S_i written
-  kBarPFull = 11,  // [2] per slot: P_i written and O_i rescaled (128 arrivals)
-  kBarODone = 13,  // [2] per slot: PV_i finished
-  kBarDrain = 15,
+  kBarP0 = 11,     // [2] per slot: P_i keys 0..63 written, O_i rescaled (128 arrivals)
+  kBarP1 = 13,     // [2] per slot: P_i keys 64..127 written (128 arrivals)
+  kBarODone = 15,  // [2] per slot: PV_i finished
+  kBarDrain = 17,  // used only when giving up
 };
 
 struct Params {
@@ -128,6 +149,37 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
+// Max over 32 values held as bit patterns (3-input max, 16 ops, two chains).
+__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
+  float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+  float b = fmax3(__uint_as_float(v[3]), __uint_as_float(v[4]), __uint_as_float(v[5]));
+#pragma unroll
+  for (int e = 6; e < 30; e += 4) {
+    a = fmax3(a, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+    b = fmax3(b, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+  }
+  return fmax3(a, b, fmaxf(__uint_as_float(v[30]), __uint_as_float(v[31])));
+}
+
+// p = 2^(s * c - mu) for 32 consecutive scores (bit patterns in v); the 16 truncated bf16
+// pairs go to out[0..15]; fp32 and truncated sums accumulate into acc / accr (pairs).
+__device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint32_t* out, uint64_t c2, uint64_t nmu2,
+                                          uint64_t& acc, uint64_t& accr) {
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const uint64_t y2 = ffma2(f2pack(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), c2, nmu2);
+    float y0, y1;
+    f2unpack(y2, y0, y1);
+    const float p0 = fast_exp2(y0), p1 = fast_exp2(y1);
+    acc = fadd2(acc, f2pack(p0, p1));
+    // bf16 P by truncation: one byte permute on the ALU pipe (a cvt would share the MUFU's
+    // pipe); O is normalised by the sum of exactly these truncated values.
+    const uint32_t w = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);
+    accr = fadd2(accr, f2pack(bf16lo(w), bf16hi(w)));
+    out[e] = w;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -154,10 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), 128);
+      mbar_init(bar(kBarP0 + s), 128);
+      mbar_init(bar(kBarP1 + s), 128);
       mbar_init(bar(kBarODone + s), 1);
+      mbar_init(bar(kBarDrain + s), 1);
     }
-    mbar_init(bar(kBarDrain), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -175,204 +228,254 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const uint32_t sQ[2] = {sbase + L::kQ, sbase + L::kQ + L::kTile};
-  const uint32_t sK[2] = {sbase + L::kK, sbase + L::kK + L::kTile};
-  const uint32_t sV[2] = {sbase + L::kV, sbase + L::kV + L::kTile};
-  const uint32_t colS[2] = {L::kColS0, L::kColS1};
-  const uint32_t colO[2] = {L::kColO0, L::kColO1};
+  const uint32_t sQ0 = sbase + L::kQ, sK0 = sbase + L::kK, sV0 = sbase + L::kV;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && N > 0) {
-      int k_fill[2] = {-1, -1}, v_fill[2] = {-1, -1};
-      uint32_t qbytes = 0;
-      for (int i = 0; i < 2; ++i) qbytes += it.n[i] > 0 ? (uint32_t)L::kTile : 0u;
-      mbar_arrive_expect_tx(bar(kBarQ), qbytes);
-      for (int i = 0; i < 2; ++i) {
-        if (it.n[i] == 0) continue;
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sQ[i] + c * L::kBox, &tmQ, bar(kBarQ), c * 64, it.t[i] * BM,
-                      it.b * p.Hq + it.h[i]);
-      }
-      const int zkv = it.b * p.Hkv + it.kvh;
-      for (int j = 0; j < N; ++j) {
-        const int s = j & 1;
-        const int f = j >> 1;
-        if (f > 0 && !mbar_wait(bar(kBarKEmpty + s), (f - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(kBarKFull + s), L::kTile);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK[s] + c * L::kBox, &tmK, bar(kBarKFull + s), c * 64, j * BN, zkv);
-        k_fill[s] = f;
-        if (f > 0 && !mbar_wait(bar(kBarVEmpty + s), (f - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(bar(kBarVFull + s), L::kTile);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sV[s] + c * L::kBox, &tmV, bar(kBarVFull + s), c * 64, j * BN, zkv);
-        v_fill[s] = f;
-      }
-      if (*abort_flag) {
-        // Let copies already in flight land before the CTA's shared memory is released.
-        int never = 0;
-        mbar_wait(bar(kBarQ), 0, &never, 100000000ull);
-        for (int s = 0; s < 2; ++s) {
-          if (k_fill[s] >= 0) mbar_wait(bar(kBarKFull + s), k_fill[s] & 1, &never, 100000000ull);
-          if (v_fill[s] >= 0) mbar_wait(bar(kBarVFull + s), v_fill[s] & 1, &never, 100000000ull);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && N > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
-      auto issue_s = [&](int i, int s) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(kk >> 2) * L::kBox + (uint32_t)(kk & 3) * 32u;
-          const uint64_t a = smem_desc_sw128(sQ[i] + off, 16, 1024);
-          const uint64_t b = smem_desc_sw128(sK[s] + off, 16, 1024);
-          mma_ss(tmem + colS[i], a, b, idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(bar(kBarSFull + i));
-      };
-      auto issue_pv = [&](int i, int s, int j) {
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          // V tile: 128 key rows of 128 bytes per 64-column box; MN-major B operand.
-          const uint64_t b = smem_desc_sw128(sV[s] + (uint32_t)kk * 2048u, L::kBox, 1024);
-          mma_ts(tmem + colO[i], tmem + colS[i] + (uint32_t)kk * 8u, b, idesc_pv,
-                 (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(bar(kBarODone + i));
-      };
-
-      bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKFull), 0, abort_flag);
-      if (ok) {
-        for (int i = 0; i < 2; ++i)
-          if (it.n[i] > 0) issue_s(i, 0);
-        tc_commit(bar(kBarKEmpty));
-      }
-      for (int j = 0; ok && j < N; ++j) {
-        const int s = j & 1;
-        const int s1 = (j + 1) & 1;
-        bool next_k = false;
-        if (!(ok = mbar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_flag))) break;
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Regs<D>::kControl));
+    if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
+      if (lane == 0 && N > 0) {
+        int k_fill[2] = {-1, -1}, v_fill[2] = {-1, -1};
+        uint32_t qbytes = 0;
+        for (int i = 0; i < 2; ++i) qbytes += it.n[i] > 0 ? (uint32_t)L::kTile : 0u;
+        mbar_arrive_expect_tx(bar(kBarQ), qbytes);
         for (int i = 0; i < 2; ++i) {
-          if (j < it.n[i]) {
-            if (!(ok = mbar_wait(bar(kBarPFull + i), j & 1, abort_flag))) break;
-            issue_pv(i, s, j);
-          }
-          if (j + 1 < it.n[i]) {
-            if (!next_k) {
-              if (!(ok = mbar_wait(bar(kBarKFull + s1), ((j + 1) >> 1) & 1, abort_flag))) break;
-              next_k = true;
-            }
-            // S_i is overwritten only after PV_i(j) has read P_i from the same columns.
-            if (!(ok = mbar_wait(bar(kBarODone + i), j & 1, abort_flag))) break;
-            issue_s(i, s1);
+          if (it.n[i] == 0) continue;
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ0 + i * L::kTile + c * L::kBox, &tmQ, bar(kBarQ), c * 64, it.t[i] * BM,
+                        it.b * p.Hq + it.h[i]);
+        }
+        const int zkv = it.b * p.Hkv + it.kvh;
+        for (int j = 0; j < N; ++j) {
+          const int s = j & 1;
+          const int f = j >> 1;
+          if (f > 0 && !mbar_wait(bar(kBarKEmpty + s), (f - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(kBarKFull + s), L::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sK0 + s * L::kTile + c * L::kBox, &tmK, bar(kBarKFull + s), c * 64, j * BN, zkv);
+          k_fill[s] = f;
+          if (f > 0 && !mbar_wait(bar(kBarVEmpty + s), (f - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(bar(kBarVFull + s), L::kTile);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sV0 + s * L::kTile + c * L::kBox, &tmV, bar(kBarVFull + s), c * 64, j * BN, zkv);
+          v_fill[s] = f;
+        }
+        if (*abort_flag) {
+          // Let copies already in flight land before the CTA's shared memory is released.
+          int never = 0;
+          mbar_wait(bar(kBarQ), 0, &never, 100000000ull);
+          for (int s = 0; s < 2; ++s) {
+            if (k_fill[s] >= 0) mbar_wait(bar(kBarKFull + s), k_fill[s] & 1, &never, 100000000ull);
+            if (v_fill[s] >= 0) mbar_wait(bar(kBarVFull + s), v_fill[s] & 1, &never, 100000000ull);
           }
         }
-        if (!ok) break;
-        tc_commit(bar(kBarVEmpty + s));
-        if (j + 1 < N) tc_commit(bar(kBarKEmpty + s1));
       }
-      if (!ok) {
-        int never = 0;
-        tc_commit(bar(kBarDrain));
-        mbar_wait(bar(kBarDrain), 0, &never, 100000000ull);
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      // Pipe order per KV tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1).  tcgen05 MMAs from one
+      // thread execute in issue order, so S_i(j+1) may be issued right behind PV_i(j), which
+      // reads P_i from the same TMEM columns.  While softmax 0 works on S_0(j+1) the pipe runs
+      // slot 1's PV and S, and the other way round.
+      if (lane == 0 && N > 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
+        auto issue_s = [&](int i, int s) {
+          tc_fence_after();
+          const uint32_t sQ = sQ0 + i * L::kTile, sK = sK0 + s * L::kTile;
+          const uint32_t tS = tmem + (i ? L::kColS1 : L::kColS0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (uint32_t)(kk >> 2) * L::kBox + (uint32_t)(kk & 3) * 32u;
+            mma_ss(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idesc_qk,
+                   kk > 0 ? 1u : 0u);
+          }
+          tc_commit(bar(kBarSFull + i));
+        };
+        // V tile: 128 key rows of 128 bytes per 64-column box; MN-major B operand.
+        auto issue_pv = [&](int i, int s, int j, int k0) {
+          tc_fence_after();
+          const uint32_t sV = sV0 + s * L::kTile;
+          const uint32_t tS = tmem + (i ? L::kColS1 : L::kColS0), tO = tmem + (i ? L::kColO1 : L::kColO0);
+#pragma unroll
+          for (int kk = k0; kk < k0 + 4; ++kk)
+            mma_ts(tO, tS + (uint32_t)kk * 8u, smem_desc_sw128(sV + (uint32_t)kk * 2048u, L::kBox, 1024), idesc_pv,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+        };
+        bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKFull), 0, abort_flag);
+        if (ok) {
+          for (int i = 0; i < 2; ++i)
+            if (it.n[i] > 0) issue_s(i, 0);
+          tc_commit(bar(kBarKEmpty));
+        }
+        for (int j = 0; ok && j < N; ++j) {
+          const int s = j & 1, s1 = (j + 1) & 1;
+          bool next_k = false;
+          if (!(ok = mbar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_flag))) break;
+          for (int i = 0; i < 2; ++i) {
+            const int ni = i ? it.n[1] : it.n[0];
+            if (j >= ni) continue;
+            if (!(ok = mbar_wait(bar(kBarP0 + i), j & 1, abort_flag))) break;
+            issue_pv(i, s, j, 0);
+            if (!(ok = mbar_wait(bar(kBarP1 + i), j & 1, abort_flag))) break;
+            issue_pv(i, s, j, 4);
+            tc_commit(bar(kBarODone + i));
+            if (j + 1 < ni) {
+              if (!next_k) {
+                if (!(ok = mbar_wait(bar(kBarKFull + s1), ((j + 1) >> 1) & 1, abort_flag))) break;
+                next_k = true;
+              }
+              issue_s(i, s1);
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar(kBarVEmpty + s));
+          if (j + 1 < N) tc_commit(bar(kBarKEmpty + s1));
+        }
+        if (!ok) {
+          int never = 0;
+          tc_commit(bar(kBarDrain));
+          mbar_wait(bar(kBarDrain), 0, &never, 100000000ull);
+        }
       }
     }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(Regs<D>::kSoftmax));
     // ------------------------------------------------------------ softmax warpgroups
-    const int i = (warp - 2) >> 2;  // slot
+    const int i = (warp - 4) >> 2;  // slot
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int n = it.n[i];
-    const int t = it.t[i];
+    const int n = i ? it.n[1] : it.n[0];
+    const int t = i ? it.t[1] : it.t[0];
+    const int h = i ? it.h[1] : it.h[0];
     if (t < p.nq) {
       const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      const uint32_t tS = tmem + lane_off + colS[i];
-      const uint32_t tO = tmem + lane_off + colO[i];
+      const uint32_t tS = tmem + lane_off + (i ? L::kColS1 : L::kColS0);
+      const uint32_t tO = tmem + lane_off + (i ? L::kColO1 : L::kColO0);
+      const uint32_t bar_s = bar(kBarSFull + i), bar_o = bar(kBarODone + i);
+      const uint32_t bar_p0 = bar(kBarP0 + i), bar_p1 = bar(kBarP1 + i);
       const int qrow = t * BM + row;
       const long long key_limit = p.causal ? (long long)qrow + p.Sk - p.Sq : (long long)p.Sk - 1;
       const long long tile_limit = p.causal ? (long long)t * BM + p.Sk - p.Sq : (long long)p.Sk - 1;
       const float c = p.scale_log2;
-      // l: fp32 row sum (for the LSE); lr: row sum of the bf16-rounded P that the tensor
-      // core multiplies, so that O / lr uses exactly normalised weights.
+      const uint64_t c2 = f2pack(c, c);
+      // l: fp32 row sum (for the LSE); lr: row sum of the bf16 P that the tensor core
+      // multiplies, so that O / lr uses exactly normalised weights.
       float m = -INFINITY, l = 0.f, lr = 0.f;
       bool ok = true;
       for (int j = 0; j < n; ++j) {
-        if (!(ok = warp_wait(bar(kBarSFull + i), j & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar_s, j & 1, abort_flag))) break;
         tc_fence_after();
-        uint32_t r[4][32];
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32u * q4, r[q4]);
-        tmem_wait_ld();
         const int kv0 = j * BN;
         // Mask only tiles that reach past the last key or the causal diagonal.
-        if ((long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk) {
+        const bool masked = (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk;
+        auto mask_chunk = [&](uint32_t(&v)[32], int q4) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int key = kv0 + q4 * 32 + e;
-              if ((long long)key > key_limit || key >= p.Sk) r[q4][e] = __float_as_uint(-INFINITY);
-            }
-        }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[q4][e]));
-        const float m_new = fmaxf(m, mx * c);
-        float alpha = 1.f;
-        if (m_new > m + kRescaleThreshold) {  // also taken on the first finite max
-          alpha = fast_exp2(m - m_new);
-          m = m_new;
-        }
-        const float mu = (m == -INFINITY) ? 0.f : m;
-        float sum = 0.f, sum_r = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[q4][2 * e]), c, -mu));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(r[q4][2 * e + 1]), c, -mu));
-            sum += p0 + p1;
-            const uint32_t w = pack_bf16x2(p0, p1);
-            sum_r += bf16lo(w) + bf16hi(w);
-            r[q4 >> 1][(q4 & 1) * 16 + e] = w;
+          for (int e = 0; e < 32; ++e) {
+            const int key = kv0 + q4 * 32 + e;
+            if ((long long)key > key_limit || key >= p.Sk) v[e] = __float_as_uint(-INFINITY);
           }
-        }
-        l = l * alpha + sum;
-        lr = lr * alpha + sum_r;
-        // P (bf16 pairs) overwrites the first 64 columns of S_i.
-        tmem_st32(tS, r[0]);
-        tmem_st32(tS + 32u, r[1]);
-        tmem_wait_st();
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          if (!(ok = warp_wait(bar(kBarODone + i), (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c4 = 0; c4 < D / 32; ++c4) {
-            uint32_t ov[32];
-            tmem_ld32(tO + 32u * c4, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(tO + 32u * c4, ov);
-          }
+        };
+        auto publish = [&](const uint32_t(&w)[32], uint32_t col, uint32_t b) {
+          tmem_st32(tS + col, w);
           tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(b);
+        };
+        uint32_t r0[32], r1[32], r2[32], r3[32], pa[32];
+        uint64_t acc0 = 0ull, accr0 = 0ull, acc1 = 0ull, accr1 = 0ull;
+        float alpha = 1.f;
+        bool fast = !__any_sync(0xffffffffu, m == -INFINITY);
+        if (fast) {
+          // Keys 0..63 against the current reference while keys 64..127 load.
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32u, r1);
+          tmem_wait_ld();
+          tmem_ld32(tS + 64u, r2);
+          tmem_ld32(tS + 96u, r3);
+          if (masked) {
+            mask_chunk(r0, 0);
+            mask_chunk(r1, 1);
+          }
+          const uint64_t nmu2 = f2pack(-m, -m);
+          exp_chunk(r0, pa, c2, nmu2, acc0, accr0);
+          exp_chunk(r1, pa + 16, c2, nmu2, acc0, accr0);
+          tmem_wait_ld();
+          if (masked) {
+            mask_chunk(r2, 2);
+            mask_chunk(r3, 3);
+          }
+          float s_lo, s_hi;
+          f2unpack(acc0, s_lo, s_hi);
+          const float mx_hi = fmaxf(max32(r2), max32(r3));
+          const bool safe = (s_lo + s_hi <= 1.8446744e19f) && (mx_hi * c <= m + kFastBound);
+          fast = !__any_sync(0xffffffffu, !safe);
+          if (fast) {
+            publish(pa, 0u, bar_p0);
+            exp_chunk(r2, r0, c2, nmu2, acc1, accr1);
+            exp_chunk(r3, r0 + 16, c2, nmu2, acc1, accr1);
+            publish(r0, 32u, bar_p1);
+          }
         }
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + i));
+        if (!fast) {
+          // First tile of a row, or a tile that may overflow the fast path: full row max.
+          tmem_ld32(tS, r0);
+          tmem_ld32(tS + 32u, r1);
+          tmem_ld32(tS + 64u, r2);
+          tmem_ld32(tS + 96u, r3);
+          tmem_wait_ld();
+          if (masked) {
+            mask_chunk(r0, 0);
+            mask_chunk(r1, 1);
+            mask_chunk(r2, 2);
+            mask_chunk(r3, 3);
+          }
+          const float mx = fmaxf(fmaxf(max32(r0), max32(r1)), fmaxf(max32(r2), max32(r3)));
+          const float m_new = fmaxf(m, mx * c);
+          if (m_new > m + kRescaleThreshold) {  // also taken on the first finite max
+            alpha = fast_exp2(m - m_new);
+            m = m_new;
+          }
+          const float mu = (m == -INFINITY) ? 0.f : m;
+          const uint64_t nmu2 = f2pack(-mu, -mu);
+          acc0 = accr0 = 0ull;
+          exp_chunk(r0, pa, c2, nmu2, acc0, accr0);
+          exp_chunk(r1, pa + 16, c2, nmu2, acc0, accr0);
+          if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // O_i must hold PV_i(j-1) before it is rescaled, and be rescaled before PV_i(j).
+            if (!(ok = warp_wait(bar_o, (j - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            const uint64_t a2 = f2pack(alpha, alpha);
+#pragma unroll
+            for (int c4 = 0; c4 < D / 32; ++c4) {
+              uint32_t ov[32];
+              tmem_ld32(tO + 32u * c4, ov);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                float o0, o1;
+                f2unpack(fmul2(f2pack(__uint_as_float(ov[2 * e]), __uint_as_float(ov[2 * e + 1])), a2), o0, o1);
+                ov[2 * e] = __float_as_uint(o0);
+                ov[2 * e + 1] = __float_as_uint(o1);
+              }
+              tmem_st32(tO + 32u * c4, ov);
+            }
+          }
+          publish(pa, 0u, bar_p0);
+          exp_chunk(r2, r0, c2, nmu2, acc1, accr1);
+          exp_chunk(r3, r0 + 16, c2, nmu2, acc1, accr1);
+          publish(r0, 32u, bar_p1);
+        }
+        float s_lo, s_hi, q_lo, q_hi;
+        f2unpack(fadd2(acc0, acc1), s_lo, s_hi);
+        f2unpack(fadd2(accr0, accr1), q_lo, q_hi);
+        l = fmaf(l, alpha, s_lo + s_hi);
+        lr = fmaf(lr, alpha, q_lo + q_hi);
       }
       // ---------------------------------------------------------- epilogue
-      if (ok && n > 0) ok = warp_wait(bar(kBarODone + i), (n - 1) & 1, abort_flag);
+      if (ok && n > 0) ok = warp_wait(bar_o, (n - 1) & 1, abort_flag);
       if (ok) {
         tc_fence_after();
-        const int bh = it.b * p.Hq + it.h[i];
+        const int bh = it.b * p.Hq + h;
         const bool in_range = qrow < p.Sq;
         const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
         __nv_bfloat16* orow =

@@ -64,13 +64,13 @@ int attn_abi_version(void);
  * D must be 64 or 128.  dtype ATTN_BF16 runs the tensor-core kernel (tcgen05 MMAs
  * with TMEM accumulators, TMA-fed tiles of 128 queries x 128 keys); q, k, v and o
  * must be 16-byte aligned.  dtype ATTN_F32 runs a CUDA-core kernel with fp32
- * arithmetic throughout (the 1e-4 accuracy path).  scale multiplies Q K^T (the pages
- * use 1/sqrt(D)).  Returns ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_HEADS,
+ * arithmetic throughout (the 1e-4 accuracy path).  scale multiplies Q K^T and must be
+ * finite and positive (the pages use 1/sqrt(D)).  Returns ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_HEADS,
  * ATTN_ERR_UNSUPPORTED or ATTN_ERR_CUDA (launch failure).  Sizes are validated on
  * the host; Sq == 0 or Sk == 0 is allowed (Sk == 0 writes O = 0, LSE = -inf).  q and o
  * may be NULL only when Sq == 0, k and v only when Sk == 0.  O is normalised by the
- * row sum of the bf16-rounded probabilities that multiply V (so the weights sum to
- * one exactly); LSE uses the unrounded fp32 row sum.
+ * row sum of the bf16 probabilities that multiply V (so the weights sum to
+ * one exactly; P is truncated to bf16); LSE uses the unrounded fp32 row sum.
  */
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
@@ -98,9 +98,14 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  * workspace.  The work is split along the KV length into chunks (attn_decode_plan);
  * each split writes a partial (O, LSE) into `workspace` and a combine pass merges
  * them with the same LSE-weighted rule as the pages' two-way online-softmax merge.
- * workspace must be device memory of at least attn_decode_workspace_bytes(...) bytes,
- * 256-byte aligned, and zero-filled before its first use; the library keeps a sticky
- * error word at its start (read and cleared by attn_decode_check).  Device-side
+ * The last split of a (sequence, head group) to finish performs that merge, so one
+ * kernel launch does the whole decode; a sequence that fits one split is written
+ * directly.  workspace must be device memory of at least
+ * attn_decode_workspace_bytes(...) bytes, 256-byte aligned, and zero-filled before its
+ * first use: it holds a sticky error word (read and cleared by attn_decode_check),
+ * per-group split counters that each call returns to zero, and the partials.  After a
+ * call that raised ATTN_DEV_WAIT_TIMEOUT, zero it again.  Calls that share a workspace
+ * must not run concurrently.  Device-side
  * checks: a block id outside [0, num_blocks), a seqlen above max_seqlen or above
  * max_blocks*block_size sets that word; the offending tokens are skipped (never
  * read) and the outputs of that sequence are unspecified.  D must be 64 or 128,
@@ -121,7 +126,7 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen
 /* Split-KV plan (pure host function, no device access):
  *   G          = largest of 8, 4, 2, 1 dividing g = Hq/Hkv (query heads per CTA);
  *   streams    = B * Hkv * (g / G);
- *   splits     = clamp(ceil(2368 / streams), 1, max(1, ceil(max_seqlen / 256)));
+ *   splits     = clamp(ceil(2368 / streams), 1, min(128, max(1, ceil(max_seqlen / 256))));
  *   chunk      = max(64, 64 * ceil(ceil(max(max_seqlen,1) / splits) / 64)) tokens;
  *   max_splits = max(1, ceil(max_seqlen / chunk)).
  * Sequence b uses ceil(seqlens[b] / chunk) splits (0 when empty).  Any output pointer
@@ -149,6 +154,13 @@ int attn_device_status(int clear, void* stream);
  * kernel then raises ATTN_DEV_WAIT_TIMEOUT in the device status and returns; it
  * never traps.  Returns the launch status. */
 int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
+
+/* Test hook for the FMA-pipe exp2 the prefill kernel uses for part of its
+ * exponentials: y[i] = 2^x[i] by range reduction to [-1/2, 1/2] and a degree-3
+ * minimax polynomial (max relative error 7.5e-5 for x >= -126; below that the result
+ * is a tiny positive number).  x and y are n floats of device memory.  Returns the
+ * launch status. */
+int attn_selftest_exp2_poly(const float* x, float* y, int n, void* stream);
 
 /* ------------------------------------------------------------------ KV-cache sizing
  * Bytes of a dense K+V cache: 2 * layers * kv_heads * head_dim * tokens * batch *

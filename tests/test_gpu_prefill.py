@@ -134,3 +134,16 @@ def test_full_size_long_context_spiked_sampled(cuda_lib):
 
 def test_no_device_error_raised(cuda_lib):
     assert device_status(clear=True) == 0
+
+
+def test_polynomial_exp2_against_exp2(cuda_lib):
+    from exact_attention_137_b200 import _lib
+
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.tensor([0.0, -0.5, 0.5, 1.0, -1.0, 7.99])])
+    y = _lib.selftest_exp2_poly(x.cuda()).cpu().double().numpy()
+    ref = np.exp2(x.double().numpy())
+    rel = np.abs(y - ref) / ref
+    assert rel.max() <= 8e-5, rel.max()
+    # below the clamp: tiny, positive, finite
+    z = _lib.selftest_exp2_poly(torch.tensor([-200.0, -1e30, -127.5], device="cuda")).cpu()
+    assert torch.all(z >= 0) and torch.all(z < 1e-37)

@@ -77,9 +77,11 @@ def test_decode_plan_bit_exact_vs_restatement(lib):
 
 def test_decode_workspace_bytes_formula(lib):
     for B, hq, hkv, d, L in [(16, 32, 8, 128, 4096), (64, 32, 8, 128, 8192), (1, 4, 1, 64, 10)]:
-        chunk, ms, _ = oracle.decode_plan_ref(B, hq, hkv, L)
-        lse_bytes = -(-(B * hq * ms * 4) // 256) * 256
-        assert _lib.decode_workspace_bytes(B, hq, hkv, d, L) == 256 + lse_bytes + B * hq * ms * d * 4
+        chunk, ms, G = oracle.decode_plan_ref(B, hq, hkv, L)
+        r256 = lambda n: -(-n // 256) * 256
+        cnt_bytes = r256(B * hkv * (hq // hkv // G) * 4)
+        lse_bytes = r256(B * hq * ms * 4)
+        assert _lib.decode_workspace_bytes(B, hq, hkv, d, L) == 256 + cnt_bytes + lse_bytes + B * hq * ms * d * 4
     assert _lib.decode_workspace_bytes(0, 1, 1, 64, 1) == 0
 
 
@@ -94,6 +96,8 @@ FAKE = ctypes.c_void_p(1 << 20)  # never dereferenced: every call below fails va
     (dict(D=96), _lib.ATTN_ERR_UNSUPPORTED),
     (dict(dtype=7), _lib.ATTN_ERR_UNSUPPORTED),
     (dict(scale=float("nan")), _lib.ATTN_ERR_ARG),
+    (dict(scale=0.0), _lib.ATTN_ERR_ARG),
+    (dict(scale=-0.5), _lib.ATTN_ERR_ARG),
     (dict(q=ctypes.c_void_p((1 << 20) + 8)), _lib.ATTN_ERR_ARG),  # bf16 path needs 16-byte alignment
 ])
 def test_fwd_rejects_bad_arguments_before_launch(lib, args, code):
