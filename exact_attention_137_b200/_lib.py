@@ -26,6 +26,8 @@ ATTN_ERR_UNSUPPORTED = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_DEVICE = 5
 ATTN_ERR_WORKSPACE = 6
+ATTN_ERR_SCRATCH_LIMIT = 7
+DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_BF16 = 0
 ATTN_F32 = 1
 ATTN_DEV_WAIT_TIMEOUT = 1
@@ -43,6 +45,8 @@ _SIGS = {
                           _c_int, _c_int, _vp]),
     "attn_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                              _c_int, _c_float, _vp, _size_t, _vp, _vp, _c_int, _vp]),
+    "attn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                     _c_int, _c_float, _vp, _vp, _c_int, _vp]),
     "attn_decode_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "attn_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _ip, _ip, _ip]),
     "attn_decode_check": (_c_int, [_vp, _vp]),
@@ -215,6 +219,33 @@ def attn_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None,
                          workspace.numel() * workspace.element_size(), _ptr(o), _ptr(lse), _dtype_code(q),
                          ctypes.c_void_p(_stream_ptr(stream)))
     _check(st, "attn_decode")
+    return o, lse
+
+
+def attn_decode_noalloc(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None,
+                        block_size: int | None = None, scale: float | None = None, o=None, lse=None, stream=None):
+    """Decode through ``attn_decode_noalloc``: no workspace, the library's fixed scratch instead.
+
+    For callers that cannot allocate device memory; tensors as in :func:`attn_decode`.
+    Calls on one device share the scratch and must not overlap on the GPU.
+    """
+    lib = load()
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    if block_table is None:
+        bs, max_blocks, num_blocks = k_cache.shape[2], 1, B
+    else:
+        bs = k_cache.shape[2] if block_size is None else int(block_size)
+        max_blocks, num_blocks = block_table.shape[1], k_cache.shape[0]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib.attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(block_table), bs,
+                                 max_blocks, num_blocks, int(max_seqlen), B, Hq, Hkv, D, sc, _ptr(o), _ptr(lse),
+                                 _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(st, "attn_decode_noalloc")
     return o, lse
 
 

@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libattn137.so")
 HEADER = os.path.join(ROOT, "include", "attn.h")
-SOURCES = [os.path.join(CSRC, "attn_api.cu")]
+SOURCES = [os.path.join(CSRC, "attn_api.cu"), os.path.join(CSRC, "attn_noalloc.cu")]
 DEPS = SOURCES + [HEADER] + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")]
 
 

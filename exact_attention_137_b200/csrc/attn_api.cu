@@ -242,6 +242,7 @@ const char* attn_error_string(int status) {
     case ATTN_ERR_CUDA: return "CUDA call failed";
     case ATTN_ERR_DEVICE: return "a kernel flagged a device-side error";
     case ATTN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case ATTN_ERR_SCRATCH_LIMIT: return "request needs more than the fixed decode scratch (ATTN_DECODE_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

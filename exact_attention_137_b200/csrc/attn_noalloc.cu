@@ -1,0 +1,69 @@
+// attn_decode_noalloc: the paged/contiguous decode for callers that must not allocate
+// device memory.
+//
+// attn_decode needs a caller-provided workspace (split partials, merge counters, an error
+// word).  Some callers cannot hand one over: code running where cudaMalloc is forbidden or
+// too slow to call (an allocator callback, a real-time loop that must never trigger the
+// implicit synchronisation an allocation can cause), or plugins inside a host framework
+// that owns every byte of device memory and offers no allocation hook.  For them the
+// library keeps its own scratch: a fixed-size array in device global memory, created when
+// the library is loaded on a device and held until the process exits.
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+
+namespace {
+
+constexpr size_t kScratchBytes = ATTN_DECODE_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+// The scratch itself.  In host code this name is only a handle for the runtime, not a
+// device address: the address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
+
+std::mutex g_mu;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per device.
+int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess || p == nullptr) return ATTN_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
+                                   const int* block_table, int block_size, int max_blocks, int num_blocks,
+                                   int max_seqlen, int B, int Hq, int Hkv, int D, float scale, void* o, float* lse,
+                                   int dtype, void* stream) {
+  int chunk = 0, max_splits = 0, heads_per_cta = 0;
+  const int plan = attn_decode_plan(B, Hq, Hkv, max_seqlen, &chunk, &max_splits, &heads_per_cta);
+  if (plan != ATTN_OK) return plan;
+  const size_t need = attn_decode_workspace_bytes(B, Hq, Hkv, D, max_seqlen);
+  if (need > kScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  const int st = scratch_address(&ws);
+  if (st != ATTN_OK) return st;
+  // The error word and the per-group split counters must start at zero.  A previous call
+  // leaves the counters at zero when it completes, but one that gave up may not; clear
+  // both (the first 256 bytes plus the 256-aligned counter block) on the caller's stream.
+  const size_t groups = (size_t)B * Hkv * (size_t)((Hq / Hkv) / heads_per_cta);
+  const size_t zero_bytes = 256 + ((groups * sizeof(int) + 255) & ~size_t(255));
+  if (cudaMemsetAsync(ws, 0, zero_bytes, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return attn_decode(q, k_cache, v_cache, seqlens, block_table, block_size, max_blocks, num_blocks, max_seqlen, B,
+                     Hq, Hkv, D, scale, ws, kScratchBytes, o, lse, dtype, stream);
+}

@@ -41,6 +41,7 @@ extern "C" {
 #define ATTN_ERR_CUDA 4        /* a CUDA runtime or driver call failed */
 #define ATTN_ERR_DEVICE 5      /* a kernel flagged an error (bad block id, wait timeout) */
 #define ATTN_ERR_WORKSPACE 6   /* workspace missing, misaligned or too small */
+#define ATTN_ERR_SCRATCH_LIMIT 7 /* attn_decode_noalloc: needs more than its fixed scratch */
 
 /* ------------------------------------------------------------------ element types */
 #define ATTN_BF16 0 /* bfloat16 storage, fp32 accumulation */
@@ -119,6 +120,36 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache,
                 int B, int Hq, int Hkv, int D, float scale,
                 void* workspace, size_t workspace_bytes,
                 void* o, float* lse, int dtype, void* stream);
+
+/* attn_decode_noalloc: the same decode as attn_decode, for callers that cannot allocate
+ * device memory at all -- for example code running inside an allocator callback, a
+ * real-time loop that must not risk the implicit synchronisation a cudaMalloc can cause,
+ * or a plugin whose host framework owns all device memory and gives it no way to ask for
+ * a workspace.  The pages have no counterpart; this is an interface convenience.
+ *
+ * Arguments are those of attn_decode without workspace/workspace_bytes.  Instead the call
+ * uses a scratch array of ATTN_DECODE_NOALLOC_SCRATCH_BYTES (16 MiB) that lives in the
+ * library's device global memory: it exists on every GPU where the library is loaded and
+ * stays allocated until the process exits.  Nothing is allocated or freed per call.
+ *  - A request whose attn_decode_workspace_bytes(...) exceeds that size returns
+ *    ATTN_ERR_SCRATCH_LIMIT before anything is launched (split the batch instead).
+ *  - The first call on a device looks up the scratch's device address once
+ *    (cudaGetSymbolAddress) with that device current; make that first call before any
+ *    stream capture begins.
+ *  - Every call clears the error word and the merge counters at the start of the scratch
+ *    with an asynchronous memset on `stream`, then runs attn_decode on it.  All calls on a
+ *    device share the one scratch, which keeps the previous call's contents: two calls
+ *    whose GPU work overlaps (different streams, or different host threads) race and
+ *    corrupt each other's partial results.  Serialise them.
+ *  - Device-side errors (bad block ids, seqlens above max_seqlen) are reported through
+ *    attn_device_status, since the scratch's error word is not visible to the caller.
+ * Returns the codes of attn_decode, plus ATTN_ERR_SCRATCH_LIMIT. */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                        const int* seqlens, const int* block_table,
+                        int block_size, int max_blocks, int num_blocks, int max_seqlen,
+                        int B, int Hq, int Hkv, int D, float scale,
+                        void* o, float* lse, int dtype, void* stream);
 
 /* Bytes of workspace attn_decode needs for these sizes (0 on invalid arguments). */
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen);

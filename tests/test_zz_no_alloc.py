@@ -1,0 +1,53 @@
+"""attn_decode_noalloc: decode without a caller workspace, for callers that cannot allocate.
+
+Some callers have no way to hand the library device memory (an allocator callback, a
+loop that must never allocate, a plugin whose host framework owns all device memory).
+For them ``attn_decode_noalloc`` runs the same decode on a fixed scratch array owned by
+the library.  These tests call it through the C ABI and compare it with ``attn_decode``
+(which uses a caller workspace) on two calls in a row, since calls share the scratch and
+each must start clean.  The file name sorts last so a stop-at-first-failure run has
+already run every other test.
+"""
+
+import pytest
+import torch
+
+from exact_attention_137_b200 import _lib
+from exact_attention_137_b200.workloads import decode_contiguous_inputs, decode_paged_inputs, to_f64
+
+from parity import BF16_TOL, compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu(x):
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in x.items()}
+
+
+@pytest.mark.parametrize("kind", ["paged", "contiguous"])
+def test_noalloc_matches_workspace_decode_on_two_calls(cuda_lib, kind):
+    if kind == "paged":
+        x = decode_paged_inputs(8, 32, 8, 128, 16, 100, 3000, seed=11, extra_blocks=3)
+    else:
+        x = decode_contiguous_inputs(6, 32, 8, 128, 2048, 1, 2048, seed=12)
+    g = _gpu(x)
+    args = dict(max_seqlen=g["max_seqlen"], block_table=g["block_table"], block_size=g["block_size"])
+    o_ref, l_ref = _lib.attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], **args)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        o, lse = _lib.attn_decode_noalloc(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], **args)
+        torch.cuda.synchronize()
+        compare(o, lse, to_f64(o_ref), to_f64(l_ref), BF16_TOL, f"noalloc {kind}")
+    assert _lib.device_status(clear=True) == 0
+
+
+def test_noalloc_rejects_requests_beyond_its_scratch(cuda_lib):
+    # 1024 sequences x 32 heads x 128 dims of fp32 partials alone exceed 16 MiB.
+    B, Hq, Hkv, D, L = 1024, 32, 8, 128, 8192
+    assert _lib.decode_workspace_bytes(B, Hq, Hkv, D, L) > _lib.DECODE_NOALLOC_SCRATCH_BYTES
+    q = torch.zeros(B, Hq, D, dtype=torch.bfloat16, device="cuda")
+    kc = torch.zeros(B, Hkv, 16, D, dtype=torch.bfloat16, device="cuda")
+    seqlens = torch.ones(B, dtype=torch.int32, device="cuda")
+    with pytest.raises(_lib.AttnError) as e:
+        _lib.attn_decode_noalloc(q, kc, kc, seqlens, max_seqlen=L)
+    assert e.value.status == _lib.ATTN_ERR_SCRATCH_LIMIT
