@@ -23,7 +23,7 @@ using attn::tc::BM;
 using attn::tc::BN;
 
 constexpr int kAbiVersion = 1;
-constexpr int kDecodeTargetCtas = 2368;
+constexpr int kDecodeTargetCtas = 1184;
 constexpr size_t kWsHeader = 256;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -144,7 +144,7 @@ bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
     }
   const long long streams = (long long)B * Hkv * (g / G);
   long long splits = cdiv(kDecodeTargetCtas, streams);
-  const long long cap = std::max(1LL, cdiv(max_seqlen, 256));
+  const long long cap = std::max(1LL, cdiv(max_seqlen, 512));
   splits = std::max(1LL, std::min(std::min(splits, cap), (long long)attn::dec::kMaxSplits));
   const long long per = cdiv(std::max(max_seqlen, 1), splits);
   const long long chunk = std::max(64LL, 64 * cdiv(per, 64));

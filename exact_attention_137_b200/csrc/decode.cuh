@@ -7,14 +7,16 @@
 //  * grid (split, kv head x head-subgroup, batch).  A CTA reads the K/V of one KV head
 //    for one chunk of tokens and serves the G query heads of its subgroup from that
 //    single read (GQA: the group's heads share each K/V row).
-//  * warp 4 streams the chunk through a 4-stage shared-memory ring with cp.async.bulk:
+//  * warp 4 streams the chunk through a 3-stage ring of 64-token stages with cp.async.bulk:
 //    every run of tokens that is contiguous in the cache (one page of a paged pool, or
 //    the whole stage in a dense cache) is one bulk copy.  The page ids come from the
 //    block table (gocoding §5), prefetched 32 pages ahead into the producer's lanes.
-//  * warps 0-3 compute.  D/8 lanes cover one 128-bit slice each of a token's row;
-//    per step each lane forms the partial dot products of D/8 (token, head) pairs and a
-//    reduce-scatter across the lane group leaves one complete score per lane.  Online
-//    softmax per head (log2 domain, ex2), then the value rows are accumulated in fp32.
+//  * warps 0-3 compute.  Eight lanes cover one token row (D/8 elements each, as
+//    interleaved 16-byte slices so that reads are conflict-free); per step
+//    each lane forms the partial dot products of 8 (token, head) pairs with packed fp32
+//    FMAs and a 3-level reduce-scatter across the 8 lanes leaves one complete score per
+//    lane (fewer lanes per row means less shuffle work per score).  Online softmax per
+//    head (log2 domain, ex2), then the value rows are accumulated as fp32 pairs.
 //  * each split writes its normalised partial output and its LSE; the combine kernel
 //    merges the splits of a (sequence, head) with weights exp(lse_s - LSE), the same
 //    two-way merge as the pages' online softmax, applied across splits.
@@ -25,8 +27,8 @@
 namespace attn {
 namespace dec {
 
-constexpr int kStageTokens = 32;
-constexpr int kStages = 4;
+constexpr int kStageTokens = 64;
+constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxSplits = 128;  // the plan never splits a sequence into more chunks
@@ -114,13 +116,19 @@ __device__ __forceinline__ float reduce_scatter(float (&vals)[LPT], int j) {
 }
 
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) {
-  constexpr int LPT = D / 8;       // lanes per token row (16 bytes each)
+__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params p) {
+  // Lanes per token row: 8, except D=128 with 8 heads per CTA, where 16 lanes halve the
+  // per-lane query and accumulator registers.
+  constexpr int LPT = (D == 128 && G == 8) ? 16 : 8;
+  constexpr int EPL = D / LPT;     // elements of a row per lane (16 at D=128, 8 at D=64)
+  constexpr int WPL = EPL / 2;     // 32-bit words (bf16 pairs) per lane per row
   constexpr int TOK = LPT / G;     // tokens per lane group per step
   constexpr int GPW = 32 / LPT;    // lane groups per warp
   constexpr int TPW = GPW * TOK;   // tokens per warp step (= 32 / G)
   constexpr int UNITS = kStageTokens / TPW;  // warp steps per stage (= G)
   static_assert(G <= LPT && TOK * G == LPT, "heads per CTA must divide the lanes per token");
+  static_assert(EPL % 8 == 0, "each lane reads whole 16-byte slices");
+  constexpr bool kJoint = true;
   using L = Layout<D>;
 
   extern __shared__ __align__(128) uint8_t smem[];
@@ -225,24 +233,32 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   }
 
   // -------------------------------------------------------------- consumers
+  // Lane j of lane group gi owns the 16-byte slices j, j + 8, ... (8 elements each) of every
+  // token row, so the 8 lanes of a group read 128 contiguous bytes per access (no bank
+  // conflicts); a group covers one row, so a score is complete after a 3-level
+  // reduce-scatter.
   const int gi = lane / LPT;
   const int j = lane - gi * LPT;
-  uint64_t q2[G][4];  // this lane's 8 query elements per head, as fp32 pairs
+  uint64_t q2[G][WPL];  // this lane's query elements per head, as fp32 pairs
 #pragma unroll
   for (int hh = 0; hh < G; ++hh) {
-    const uint4 w = __ldg(reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D) + j);
-    q2[hh][0] = f2pack(bf16lo(w.x), bf16hi(w.x));
-    q2[hh][1] = f2pack(bf16lo(w.y), bf16hi(w.y));
-    q2[hh][2] = f2pack(bf16lo(w.z), bf16hi(w.z));
-    q2[hh][3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D) + j;
+#pragma unroll
+    for (int v4 = 0; v4 < EPL / 8; ++v4) {
+      const uint4 w = __ldg(src + LPT * v4);
+      q2[hh][4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
+      q2[hh][4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
+      q2[hh][4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
+      q2[hh][4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+    }
   }
   const float c = p.scale_log2;
   float m_own = -INFINITY, l_own = 0.f;
-  uint64_t acc[G][4];
+  uint64_t acc[G][WPL];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) acc[hh][e] = 0ull;
+    for (int e = 0; e < WPL; ++e) acc[hh][e] = 0ull;
 
   bool ok = true;
   for (int it = 0; it < niters; ++it) {
@@ -252,36 +268,52 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
     const int nv = min(kStageTokens, t1 - (t0 + it * kStageTokens));
     const uint32_t sk = sbase + L::kK + s * L::kStageBytes;
     const uint32_t sv = sbase + L::kV + s * L::kStageBytes;
-    for (int u = warp; u < UNITS; u += kConsumerWarps) {
-      const int tb = u * TPW + gi * TOK;  // first token of this lane group in the stage
-      float vals[LPT];
+    // Each warp takes two units of the stage at a time (u and u + 4 warps): their dot
+    // products and reductions are independent, which gives the warp twice the ILP; they
+    // share one max update and one rescale.  A second unit past the stage is empty.
+    for (int u = warp; u < UNITS; u += (kJoint ? 2 : 1) * kConsumerWarps) {
+      const int u1 = u + kConsumerWarps;
+      const bool has1 = kJoint && u1 < UNITS;
+      const int tb0 = u * TPW + gi * TOK;                   // first token of this lane group
+      const int tb1 = (has1 ? u1 : u) * TPW + gi * TOK;
+      float vals0[LPT], vals1[LPT];
 #pragma unroll
       for (int tt = 0; tt < TOK; ++tt) {
-        const uint4 w = lds128(sk + (uint32_t)(tb + tt) * L::kRow + 16u * j);
-        const uint64_t k0 = f2pack(bf16lo(w.x), bf16hi(w.x)), k1 = f2pack(bf16lo(w.y), bf16hi(w.y));
-        const uint64_t k2 = f2pack(bf16lo(w.z), bf16hi(w.z)), k3 = f2pack(bf16lo(w.w), bf16hi(w.w));
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          uint64_t d2 = fmul2(q2[hh][0], k0);
-          d2 = ffma2(q2[hh][1], k1, d2);
-          d2 = ffma2(q2[hh][2], k2, d2);
-          d2 = ffma2(q2[hh][3], k3, d2);
-          float lo, hi;
-          f2unpack(d2, lo, hi);
-          vals[tt * G + hh] = lo + hi;
+        for (int x = 0; x < 2; ++x) {
+          uint64_t k2[WPL];
+#pragma unroll
+          for (int v4 = 0; v4 < EPL / 8; ++v4) {
+            const uint4 w = lds128(sk + (uint32_t)((x ? tb1 : tb0) + tt) * L::kRow + 16u * (j + LPT * v4));
+            k2[4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
+            k2[4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
+            k2[4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
+            k2[4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+          }
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            uint64_t d2 = fmul2(q2[hh][0], k2[0]);
+#pragma unroll
+            for (int e = 1; e < WPL; ++e) d2 = ffma2(q2[hh][e], k2[e], d2);
+            float lo, hi;
+            f2unpack(d2, lo, hi);
+            if (x) vals1[tt * G + hh] = lo + hi;
+            else vals0[tt * G + hh] = lo + hi;
+          }
         }
       }
-      const float score = reduce_scatter<LPT>(vals, j);
-      const bool valid = tb + j / G < nv;
-      const float x = valid ? score * c : -INFINITY;
-      float mx = x;
+      const float score0 = reduce_scatter<LPT>(vals0, j);
+      const float score1 = reduce_scatter<LPT>(vals1, j);
+      const float x0 = (tb0 + j / G < nv) ? score0 * c : -INFINITY;
+      const float x1 = (has1 && tb1 + j / G < nv) ? score1 * c : -INFINITY;
+      float mx = fmaxf(x0, x1);
 #pragma unroll
       for (int o = G; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
       const float m_new = fmaxf(m_own, mx);
       const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_own - m_new);
       const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-      const float pr = fast_exp2(x - mu);
-      l_own = l_own * alpha + pr;
+      const float pr0 = fast_exp2(x0 - mu), pr1 = fast_exp2(x1 - mu);
+      l_own = l_own * alpha + (pr0 + pr1);
       m_own = m_new;
       if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
@@ -289,24 +321,32 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
           const float ah = __shfl_sync(0xffffffffu, alpha, hh);
           const uint64_t a2 = f2pack(ah, ah);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[hh][e] = fmul2(acc[hh][e], a2);
+          for (int e = 0; e < WPL; ++e) acc[hh][e] = fmul2(acc[hh][e], a2);
         }
       }
 #pragma unroll
       for (int tt = 0; tt < TOK; ++tt) {
-        const uint4 w = lds128(sv + (uint32_t)(tb + tt) * L::kRow + 16u * j);
-        const uint64_t v0 = f2pack(bf16lo(w.x), bf16hi(w.x)), v1 = f2pack(bf16lo(w.y), bf16hi(w.y));
-        const uint64_t v2 = f2pack(bf16lo(w.z), bf16hi(w.z)), v3 = f2pack(bf16lo(w.w), bf16hi(w.w));
-        const bool tv = tb + tt < nv;
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const float ph = __shfl_sync(0xffffffffu, pr, gi * LPT + tt * G + hh);
-          if (tv) {
-            const uint64_t p2 = f2pack(ph, ph);
-            acc[hh][0] = ffma2(p2, v0, acc[hh][0]);
-            acc[hh][1] = ffma2(p2, v1, acc[hh][1]);
-            acc[hh][2] = ffma2(p2, v2, acc[hh][2]);
-            acc[hh][3] = ffma2(p2, v3, acc[hh][3]);
+        for (int x = 0; x < 2; ++x) {
+          uint64_t v2[WPL];
+          const int tok = (x ? tb1 : tb0) + tt;
+#pragma unroll
+          for (int v4 = 0; v4 < EPL / 8; ++v4) {
+            const uint4 w = lds128(sv + (uint32_t)tok * L::kRow + 16u * (j + LPT * v4));
+            v2[4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
+            v2[4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
+            v2[4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
+            v2[4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+          }
+          const bool tv = (x == 0 || has1) && tok < nv;
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const float ph = __shfl_sync(0xffffffffu, x ? pr1 : pr0, gi * LPT + tt * G + hh);
+            if (tv) {
+              const uint64_t p2 = f2pack(ph, ph);
+#pragma unroll
+              for (int e = 0; e < WPL; ++e) acc[hh][e] = ffma2(p2, v2[e], acc[hh][e]);
+            }
           }
         }
       }
@@ -316,17 +356,17 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
   }
 
   // Merge lane groups of this warp: per head, acc summed over groups, l over all lanes.
-  float accf[G][8];
+  float accf[G][EPL];
 #pragma unroll
   for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) f2unpack(acc[hh][e], accf[hh][2 * e], accf[hh][2 * e + 1]);
+    for (int e = 0; e < WPL; ++e) f2unpack(acc[hh][e], accf[hh][2 * e], accf[hh][2 * e + 1]);
 #pragma unroll
   for (int o = LPT; o < 32; o <<= 1)
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) accf[hh][e] += __shfl_xor_sync(0xffffffffu, accf[hh][e], o);
+      for (int e = 0; e < EPL; ++e) accf[hh][e] += __shfl_xor_sync(0xffffffffu, accf[hh][e], o);
   float l_sum = l_own;
 #pragma unroll
   for (int o = G; o < 32; o <<= 1) l_sum += __shfl_xor_sync(0xffffffffu, l_sum, o);
@@ -351,7 +391,7 @@ __global__ void __launch_bounds__(kThreads) decode_split_kernel(const Params p) 
 #pragma unroll
       for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) a_s[(warp * G + hh) * D + 8 * j + e] = accf[hh][e];
+        for (int e = 0; e < EPL; ++e) a_s[(warp * G + hh) * D + 8 * (j + LPT * (e >> 3)) + (e & 7)] = accf[hh][e];
     }
   }
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));

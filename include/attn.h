@@ -157,7 +157,7 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen
 /* Split-KV plan (pure host function, no device access):
  *   G          = largest of 8, 4, 2, 1 dividing g = Hq/Hkv (query heads per CTA);
  *   streams    = B * Hkv * (g / G);
- *   splits     = clamp(ceil(2368 / streams), 1, min(128, max(1, ceil(max_seqlen / 256))));
+ *   splits     = clamp(ceil(1184 / streams), 1, min(128, max(1, ceil(max_seqlen / 512))));
  *   chunk      = max(64, 64 * ceil(ceil(max(max_seqlen,1) / splits) / 64)) tokens;
  *   max_splits = max(1, ceil(max_seqlen / chunk)).
  * Sequence b uses ceil(seqlens[b] / chunk) splits (0 when empty).  Any output pointer

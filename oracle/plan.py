@@ -9,8 +9,8 @@ same attention result; the decode parity tests check that.
 
 * heads per CTA ``G``: the largest of 8, 4, 2, 1 that divides ``g = Hq / Hkv``;
 * independent streams ``U = B * Hkv * (g / G)``;
-* splits wanted ``ceil(TARGET_CTAS / U)`` with ``TARGET_CTAS = 2368``, clamped to
-  ``[1, min(128, max(1, ceil(max_seqlen / 256)))]``;
+* splits wanted ``ceil(TARGET_CTAS / U)`` with ``TARGET_CTAS = 1184``, clamped to
+  ``[1, min(128, max(1, ceil(max_seqlen / 512)))]``;
 * ``chunk = 64 * ceil(ceil(max_seqlen / splits) / 64)`` tokens per split (at least 64);
 * ``max_splits = max(1, ceil(max_seqlen / chunk))``;
 * sequence ``b`` uses ``ceil(seqlen_b / chunk)`` splits.
@@ -20,7 +20,7 @@ from __future__ import annotations
 
 __all__ = ["decode_plan_ref", "decode_heads_per_cta_ref", "TARGET_CTAS"]
 
-TARGET_CTAS = 2368
+TARGET_CTAS = 1184
 MAX_SPLITS = 128
 
 
@@ -44,7 +44,7 @@ def decode_plan_ref(batch: int, hq: int, hkv: int, max_seqlen: int):
     G = decode_heads_per_cta_ref(hq, hkv)
     streams = batch * hkv * (g // G)
     splits = _cdiv(TARGET_CTAS, streams)
-    splits = max(1, min(splits, max(1, _cdiv(max_seqlen, 256)), MAX_SPLITS))
+    splits = max(1, min(splits, max(1, _cdiv(max_seqlen, 512)), MAX_SPLITS))
     chunk = max(64, 64 * _cdiv(_cdiv(max(max_seqlen, 1), splits), 64))
     max_splits = max(1, _cdiv(max_seqlen, chunk))
     return chunk, max_splits, G
