@@ -6,7 +6,7 @@ One step is one pass of the whole hot path over synthetic inputs resident in HBM
 * prefill head-sharing sweep: B=2, Hq=32, Hkv in {32, 8, 1}, Sq=Sk=2048, D=128, bf16,
   causal -- three ``attn_fwd`` calls (one tensor-core kernel each);
 * paged GQA decode: B=64, Hq=32, Hkv=8, D=128, block 16, lengths U[512, 8192], pool
-  permuted -- one ``attn_decode`` call (split kernel + combine kernel);
+  permuted -- one ``attn_decode`` call (one kernel: split partials, merged by the last split);
 * contiguous GQA decode: B=16, Hq=32, Hkv=8, D=128, capacity 4096, lengths
   U[1024, 4096] -- one ``attn_decode`` call.
 
@@ -57,7 +57,7 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples every 200 ms while running."""
+    """nvidia-smi clock / throttle-reason samples every 100 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -72,7 +72,7 @@ class ClockSampler:
         try:
             self.out = tempfile.NamedTemporaryFile("w+", delete=False, suffix=".csv")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
                  "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, ValueError):
             self.proc = None
@@ -149,29 +149,56 @@ def barrier(world: int):
 
 
 def oracle_prefill_sample(target_s: float):
-    """Time the fp64 oracle on whole query heads of the GQA (Hkv=8) S=2048 causal case."""
-    import numpy as np
+    """Time the fp64 oracle on whole query heads of the prefill sweep, about target_s seconds.
 
+    Heads are taken in order over the three Hkv variants (batch 0, then batch 1) until the
+    time budget is spent; each head is exact over all its rows.
+    """
     from exact_attention_137_b200.workloads import prefill_inputs, to_f64
     from oracle import attention_ref
 
-    B, Hq, S, D = 1, 32, PREFILL["S"], PREFILL["D"]
-    x = prefill_inputs(B, Hq, 8, S, S, D, dtype="bf16", seed=0)
-    q, k, v = to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"])
-    g = Hq // 8
-    t0 = time.perf_counter()
-    attention_ref(q[:, :1], k[:, :1], v[:, :1], causal=True)
-    t1 = time.perf_counter() - t0
-    nh = int(max(1, min(Hq, round(target_s / max(t1, 1e-3)))))
-    nkv = -(-nh // g)
-    t0 = time.perf_counter()
-    attention_ref(q[:, :nh], k[:, :nkv], v[:, :nkv], causal=True)
-    dt = time.perf_counter() - t0
-    flops = prefill_flops(1, nh, S, D)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
+    S, D, Hq = PREFILL["S"], PREFILL["D"], PREFILL["Hq"]
+    done_flops, spent, heads = 0.0, 0.0, 0
+    for b in range(PREFILL["B"]):
+        for hkv in PREFILL["hkvs"]:
+            x = prefill_inputs(PREFILL["B"], Hq, hkv, S, S, D, dtype="bf16", seed=0)
+            g = Hq // hkv
+            q, k, v = to_f64(x["q"][b:b + 1]), to_f64(x["k"][b:b + 1]), to_f64(x["v"][b:b + 1])
+            for h in range(Hq):
+                if spent >= target_s:
+                    break
+                t0 = time.perf_counter()
+                attention_ref(q[:, h:h + 1], k[:, h // g:h // g + 1], v[:, h // g:h // g + 1], causal=True)
+                spent += time.perf_counter() - t0
+                done_flops += prefill_flops(1, 1, S, D)
+                heads += 1
+    return {"value": done_flops / spent / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
             "kind": "oracle",
-            "sample": f"b=0, query heads 0..{nh - 1} (all {S} rows) of the Hkv=8 S={S} D={D} causal case; "
-                      f"{dt:.1f} s; numpy fp64 with full score matrices"}
+            "sample": f"{heads} whole query heads (all {S} rows, causal) of the prefill sweep B=2 Hq=32 "
+                      f"Hkv in {{32,8,1}} D={D}, taken in order; {spent:.1f} s of numpy fp64 with full score "
+                      f"matrices; throughput counts algorithmic (unmasked) FLOPs"}
+
+
+def profile_traffic(name: str):
+    """ncu DRAM bytes per launch recorded in profiles/<name>.md, or None if the kernel source
+    has changed since that capture (the summary stores a hash of the source files)."""
+    import hashlib
+    import re
+
+    path = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(path):
+        return None
+    text = open(path, encoding="utf-8").read()
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_hash = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_files = re.search(r"source_files:\s*(.+)", text)
+    if not (m_bytes and m_hash and m_files):
+        return None
+    h = hashlib.sha256()
+    for f in m_files.group(1).split():
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return float(m_bytes.group(1)) if h.hexdigest() == m_hash.group(1) else None
 
 
 def run_reference(args, rank, world):
@@ -351,11 +378,13 @@ def run_ours(args, rank, world, local):
     per_launch_ms = pre_ms / len(pre)
     achieved_tf = fl_call / (per_launch_ms * 1e-3) / 1e12
 
-    def dec_obj(name, g, spec_name):
+    def dec_obj(name, g, spec_name, prof):
         ms = max_over_ranks(per_call[name], world)
         gbs = g["bytes"] / (ms * 1e-3) / 1e9
         return {"workload": spec_name, "ms": ms, "GB/s": gbs, "kv_bytes": g["kv_bytes"], "bytes": g["bytes"],
-                "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "kernels": ["decode_split_kernel (split partials + merge by the last split)"]}
+                "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "bound": "hbm",
+                "traffic": profile_traffic(prof),
+                "kernels": ["decode_split_kernel (split partials + merge by the last split)"]}
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -367,11 +396,15 @@ def run_ours(args, rank, world, local):
                    "prefill_flops_per_call": fl_call, "prefill_ms_per_call": {c["hkv"]: per_call["prefill_hkv%d" % c["hkv"]] for c in pre},
                    "parallelism": "replicas" if world > 1 else "single GPU"},
         "roofline": {"bound": "tensor", "kernel": "attn::tc::fwd_tc_kernel<128>", "achieved": achieved_tf,
-                     "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved_tf / tf_peak, "traffic": None,
-                     "peak_source": f"{peak_src} bf16 dense (burst)"},
-        "decode": {"paged": dec_obj("decode_paged", paged, "B=64 Hq=32 Hkv=8 D=128 block 16 len U[512,8192]"),
+                     "peak": tf_peak, "unit": "TFLOP/s", "frac": achieved_tf / tf_peak,
+                     "traffic": profile_traffic("prefill_tc_gqa_s2048"),
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "per_launch": "68.75 GFLOP (B=2, Hq=32, S=2048, D=128 causal, unmasked pairs)"},
+        "decode": {"paged": dec_obj("decode_paged", paged, "B=64 Hq=32 Hkv=8 D=128 block 16 len U[512,8192]",
+                                    "decode_split_paged_b64"),
                    "contiguous": dec_obj("decode_contiguous", contig,
-                                         "B=16 Hq=32 Hkv=8 D=128 cap 4096 len U[1024,4096]")},
+                                         "B=16 Hq=32 Hkv=8 D=128 cap 4096 len U[1024,4096]",
+                                         "decode_split_contiguous_b16")},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill sweep with q/k/v copied from pinned host memory and O/LSE copied back each step"},
         "gpu_launches": launches_per_step * args.steps,
@@ -387,11 +420,11 @@ def run_ours(args, rank, world, local):
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))
