@@ -373,6 +373,36 @@ def run_ours(args, rank, world, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world)
     e2e_value = world * len(pre) * fl_call / (e2e_ms * 1e-3) / 1e12
 
+    # Decode head-sharing sweep (context, outside the timed region): the paged workload's
+    # lengths and pool layout with Hkv in {32, 8, 1} at Hq=32, inputs drawn on the device.
+    sweep = None
+    if not args.no_decode_sweep:
+        sweep = []
+        for hkv in (32, 8, 1):
+            sx = decode_paged_inputs(S["B"], S["Hq"], hkv, S["D"], S["bs"], S["lo"], S["hi"], seed=seed, device=dev)
+            sg = decode_case(sx, dict(S, Hkv=hkv))
+            for _ in range(3):
+                flush.fill_(1.0)
+                run_decode(sg)
+            sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.sweep_iters)]
+            for i in range(args.sweep_iters):
+                flush.fill_(float(i))
+                sev[i][0].record(stream)
+                run_decode(sg)
+                sev[i][1].record(stream)
+            torch.cuda.synchronize()
+            ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in sev) / len(sev), world)
+            sweep.append({"Hkv": hkv, "ms": ms, "GB/s": sg["bytes"] / (ms * 1e-3) / 1e9,
+                          "frac": sg["bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "kv_bytes": sg["kv_bytes"], "tokens_per_s": S["B"] / (ms * 1e-3)})
+            del sx, sg
+            torch.cuda.empty_cache()
+        base = sweep[0]["tokens_per_s"]
+        for r in sweep:
+            r["relative_to_mha"] = r["tokens_per_s"] / base
+        assert device_status(clear=True) == 0
+
     hbm = peaks["hbm_gbs"]
     tf_peak = peaks["bf16_tflops"]
     per_launch_ms = pre_ms / len(pre)
@@ -384,7 +414,7 @@ def run_ours(args, rank, world, local):
         return {"workload": spec_name, "ms": ms, "GB/s": gbs, "kv_bytes": g["kv_bytes"], "bytes": g["bytes"],
                 "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "bound": "hbm",
                 "traffic": profile_traffic(prof),
-                "kernels": ["decode_split_kernel (split partials + merge by the last split)"]}
+                "kernels": ["decode_kernel (balanced split partials + merge by the last CTA of a stream)"]}
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -405,6 +435,10 @@ def run_ours(args, rank, world, local):
                    "contiguous": dec_obj("decode_contiguous", contig,
                                          "B=16 Hq=32 Hkv=8 D=128 cap 4096 len U[1024,4096]",
                                          "decode_split_contiguous_b16")},
+        "decode_sweep": None if sweep is None else {
+            "workload": "paged B=64 Hq=32 D=128 block 16 len U[512,8192], Hkv in {32 (MHA), 8 (GQA), 1 (MQA)}; "
+                        "one decoded token per sequence; L2 flushed before each call",
+            "rows": sweep},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill sweep with q/k/v copied from pinned host memory and O/LSE copied back each step"},
         "gpu_launches": launches_per_step * args.steps,
@@ -424,6 +458,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode-sweep", action="store_true")
+    ap.add_argument("--sweep-iters", type=int, default=30)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.impl == "reference":

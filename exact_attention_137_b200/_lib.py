@@ -48,7 +48,8 @@ _SIGS = {
     "attn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_int, _c_float, _vp, _vp, _c_int, _vp]),
     "attn_decode_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
-    "attn_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _ip, _ip, _ip]),
+    "attn_decode_plan": (_c_int, [_c_int, _c_int, _c_int, _c_int, _c_int, _ip, _ip]),
+    "attn_decode_schedule": (_c_int, [_ip, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _ip, _c_int, _ip]),
     "attn_decode_check": (_c_int, [_vp, _vp]),
     "attn_device_status": (_c_int, [_c_int, _vp]),
     "attn_selftest_wait_timeout": (_c_int, [_ull, _vp]),
@@ -155,12 +156,26 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
 # ------------------------------------------------------------------ decode
 
 
-def decode_plan(B: int, Hq: int, Hkv: int, max_seqlen: int):
+def decode_plan(B: int, Hq: int, Hkv: int, max_seqlen: int, num_sms: int):
+    """``(ctas, heads_per_cta)`` of a decode launch on a device with ``num_sms`` SMs."""
     lib = load()
-    c, m, g = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(lib.attn_decode_plan(B, Hq, Hkv, max_seqlen, ctypes.byref(c), ctypes.byref(m), ctypes.byref(g)),
+    c, g = ctypes.c_int(), ctypes.c_int()
+    _check(lib.attn_decode_plan(B, Hq, Hkv, max_seqlen, num_sms, ctypes.byref(c), ctypes.byref(g)),
            "attn_decode_plan")
-    return c.value, m.value, g.value
+    return c.value, g.value
+
+
+def decode_schedule(seqlens, Hq: int, Hkv: int, max_seqlen: int, ctas: int, cta: int):
+    """Segments of CTA ``cta`` as tuples ``(b, y, tok0, tok1, slot, nsplit)`` (host-side listing)."""
+    lib = load()
+    lens = (ctypes.c_int * len(seqlens))(*[int(x) for x in seqlens])
+    n = ctypes.c_int()
+    _check(lib.attn_decode_schedule(lens, len(seqlens), Hq, Hkv, max_seqlen, ctas, cta, None, 0, ctypes.byref(n)),
+           "attn_decode_schedule")
+    buf = (ctypes.c_int * (6 * max(1, n.value)))()
+    _check(lib.attn_decode_schedule(lens, len(seqlens), Hq, Hkv, max_seqlen, ctas, cta, buf, n.value,
+                                    ctypes.byref(n)), "attn_decode_schedule")
+    return [tuple(buf[6 * i:6 * i + 6]) for i in range(n.value)]
 
 
 def decode_workspace_bytes(B: int, Hq: int, Hkv: int, D: int, max_seqlen: int) -> int:

@@ -22,8 +22,7 @@ namespace {
 using attn::tc::BM;
 using attn::tc::BN;
 
-constexpr int kAbiVersion = 1;
-constexpr int kDecodeTargetCtas = 1184;
+constexpr int kAbiVersion = 2;
 constexpr size_t kWsHeader = 256;
 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -130,7 +129,7 @@ int launch_fwd_simt(const void* q, const void* k, const void* v, void* o, float*
 }
 
 struct DecodePlan {
-  int chunk, max_splits, G;
+  int G, Y, ctas_cap;  // heads per CTA, streams per sequence, CTA bound from the sizes alone
 };
 
 bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
@@ -142,40 +141,55 @@ bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
       G = cand;
       break;
     }
-  const long long streams = (long long)B * Hkv * (g / G);
-  long long splits = cdiv(kDecodeTargetCtas, streams);
-  const long long cap = std::max(1LL, cdiv(max_seqlen, 512));
-  splits = std::max(1LL, std::min(std::min(splits, cap), (long long)attn::dec::kMaxSplits));
-  const long long per = cdiv(std::max(max_seqlen, 1), splits);
-  const long long chunk = std::max(64LL, 64 * cdiv(per, 64));
-  out->chunk = (int)chunk;
-  out->max_splits = (int)std::max(1LL, cdiv(max_seqlen, chunk));
+  const long long Y = (long long)Hkv * (g / G);
+  const long long umax = (long long)B * Y * attn::dec::units_of(max_seqlen);
+  if (umax >= (1LL << 52)) return false;  // keeps i * total and (x + 1) * n within 64 bits
   out->G = G;
+  out->Y = (int)Y;
+  out->ctas_cap = (int)std::min<long long>(attn::dec::kMaxCtas,
+                                           std::max(1LL, cdiv(umax, attn::dec::kMinUnitsPerCta)));
   return true;
+}
+
+inline int plan_ctas(const DecodePlan& pl, int num_sms) {
+  return std::max(1, std::min(pl.ctas_cap, attn::dec::kCtasPerSm * std::max(1, num_sms)));
+}
+
+// SM count of the current device, looked up once per device.
+int device_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    sms[dev] = v;
+  }
+  return sms[dev];
 }
 
 inline size_t round256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace layout: [error word | 256 B] [split counters, B*Hkv*(g/G) int32, 256-aligned]
-// [partial LSE, B*Hq*max_splits fp32, 256-aligned] [partial O, B*Hq*max_splits*D fp32].
+// Workspace layout: [error word | 256 B] [merge counters, B*Y int32, 256-aligned]
+// [partial LSE, ctas_cap*2*G fp32, 256-aligned] [partial O, ctas_cap*2*G*D fp32].
 struct WsLayout {
   size_t cnt, lse, o, total;
 };
 
-WsLayout ws_layout(int B, int Hq, int Hkv, int D, const DecodePlan& pl) {
+WsLayout ws_layout(int B, int D, const DecodePlan& pl) {
   WsLayout w;
-  const size_t streams = (size_t)B * Hkv * ((Hq / Hkv) / pl.G);
+  const size_t slots = (size_t)pl.ctas_cap * 2 * pl.G;
   w.cnt = kWsHeader;
-  w.lse = w.cnt + round256(streams * sizeof(int));
-  w.o = w.lse + round256((size_t)B * Hq * pl.max_splits * sizeof(float));
-  w.total = w.o + (size_t)B * Hq * pl.max_splits * D * sizeof(float);
+  w.lse = w.cnt + round256((size_t)B * pl.Y * sizeof(int));
+  w.o = w.lse + round256(slots * sizeof(float));
+  w.total = w.o + slots * D * sizeof(float);
   return w;
 }
 
 template <int D, int G>
-int launch_decode_split(const attn::dec::Params& p, cudaStream_t st) {
-  using Lay = attn::dec::Layout<D>;
-  auto kern = attn::dec::decode_split_kernel<D, G>;
+int launch_decode(const attn::dec::Params& p, int ctas, cudaStream_t st) {
+  using Lay = attn::dec::Layout<D, G>;
+  auto kern = attn::dec::decode_kernel<D, G>;
   const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3);
   static bool done[64][8] = {};
   static std::mutex mu;
@@ -189,18 +203,17 @@ int launch_decode_split(const attn::dec::Params& p, cudaStream_t st) {
       done[dev][key] = true;
     }
   }
-  dim3 grid((unsigned)p.max_splits, (unsigned)(p.Hkv * p.nsub), (unsigned)p.B);
-  kern<<<grid, attn::dec::kThreads, Lay::kBytes, st>>>(p);
+  kern<<<(unsigned)ctas, attn::dec::kThreads, Lay::kBytes, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D>
-int dispatch_decode_g(const attn::dec::Params& p, int G, cudaStream_t st) {
+int dispatch_decode_g(const attn::dec::Params& p, int G, int ctas, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode_split<D, 1>(p, st);
-    case 2: return launch_decode_split<D, 2>(p, st);
-    case 4: return launch_decode_split<D, 4>(p, st);
-    case 8: return launch_decode_split<D, 8>(p, st);
+    case 1: return launch_decode<D, 1>(p, ctas, st);
+    case 2: return launch_decode<D, 2>(p, ctas, st);
+    case 4: return launch_decode<D, 4>(p, ctas, st);
+    case 8: return launch_decode<D, 8>(p, ctas, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
@@ -278,22 +291,54 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
                  : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st);
 }
 
-int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int* chunk_tokens, int* max_splits,
-                     int* heads_per_cta) {
+int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int num_sms, int* ctas, int* heads_per_cta) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_seqlen < 0) return ATTN_ERR_ARG;
   if (Hq % Hkv) return ATTN_ERR_HEADS;
   DecodePlan pl;
   if (!decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return ATTN_ERR_ARG;
-  if (chunk_tokens) *chunk_tokens = pl.chunk;
-  if (max_splits) *max_splits = pl.max_splits;
+  if (ctas) *ctas = plan_ctas(pl, num_sms);
   if (heads_per_cta) *heads_per_cta = pl.G;
+  return ATTN_OK;
+}
+
+int attn_decode_schedule(const int* seqlens_host, int B, int Hq, int Hkv, int max_seqlen, int ctas, int cta,
+                         int* segs, int max_segs, int* nseg) {
+  if (!seqlens_host || !nseg || ctas <= 0 || cta < 0 || cta >= ctas || max_segs < 0 || (max_segs > 0 && !segs))
+    return ATTN_ERR_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || max_seqlen < 0) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  DecodePlan pl;
+  if (!decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return ATTN_ERR_ARG;
+  const attn::dec::HostLens len_of{seqlens_host, max_seqlen};
+  long long total = 0;
+  for (int b = 0; b < B; ++b) total += attn::dec::units_of(len_of(b));
+  total *= pl.Y;
+  *nseg = 0;
+  const int n = attn::dec::active_ctas(total, ctas);
+  if (cta >= n) return ATTN_OK;
+  attn::dec::Walk w = attn::dec::walk_start_host(len_of, B, pl.Y, total, n, cta);
+  attn::dec::Segment sg;
+  int k = 0;
+  while (attn::dec::next_segment(w, len_of, pl.Y, total, n, sg)) {
+    if (k < max_segs) {
+      int* r = segs + 6 * (size_t)k;
+      r[0] = sg.b;
+      r[1] = sg.y;
+      r[2] = sg.tok0;
+      r[3] = sg.tok1;
+      r[4] = sg.slot;
+      r[5] = sg.nsplit;
+    }
+    ++k;
+  }
+  *nseg = k;
   return ATTN_OK;
 }
 
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen) {
   DecodePlan pl;
   if (D <= 0 || !decode_plan(B, Hq, Hkv, max_seqlen, &pl)) return 0;
-  return ws_layout(B, Hq, Hkv, D, pl).total;
+  return ws_layout(B, D, pl).total;
 }
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
@@ -333,11 +378,11 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.chunk = pl.chunk;
-  p.max_splits = pl.max_splits;
   p.nsub = (Hq / Hkv) / pl.G;
   p.scale_log2 = scale * attn::kLog2e;
-  const WsLayout wl = ws_layout(B, Hq, Hkv, D, pl);
+  const WsLayout wl = ws_layout(B, D, pl);
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
   p.ws_err = reinterpret_cast<unsigned int*>(ws);
   p.ws_cnt = reinterpret_cast<int*>(ws + wl.cnt);
   p.ws_lse = reinterpret_cast<float*>(ws + wl.lse);
@@ -345,7 +390,8 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   cudaStream_t st = as_stream(stream);
-  return D == 64 ? dispatch_decode_g<64>(p, pl.G, st) : dispatch_decode_g<128>(p, pl.G, st);
+  const int ctas = plan_ctas(pl, sms);
+  return D == 64 ? dispatch_decode_g<64>(p, pl.G, ctas, st) : dispatch_decode_g<128>(p, pl.G, ctas, st);
 }
 
 int attn_decode_check(void* workspace, void* stream) {

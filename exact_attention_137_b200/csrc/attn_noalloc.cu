@@ -50,15 +50,15 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
                                    const int* block_table, int block_size, int max_blocks, int num_blocks,
                                    int max_seqlen, int B, int Hq, int Hkv, int D, float scale, void* o, float* lse,
                                    int dtype, void* stream) {
-  int chunk = 0, max_splits = 0, heads_per_cta = 0;
-  const int plan = attn_decode_plan(B, Hq, Hkv, max_seqlen, &chunk, &max_splits, &heads_per_cta);
+  int heads_per_cta = 0;
+  const int plan = attn_decode_plan(B, Hq, Hkv, max_seqlen, 1, nullptr, &heads_per_cta);
   if (plan != ATTN_OK) return plan;
   const size_t need = attn_decode_workspace_bytes(B, Hq, Hkv, D, max_seqlen);
   if (need > kScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
   void* ws = nullptr;
   const int st = scratch_address(&ws);
   if (st != ATTN_OK) return st;
-  // The error word and the per-group split counters must start at zero.  A previous call
+  // The error word and the per-stream merge counters must start at zero.  A previous call
   // leaves the counters at zero when it completes, but one that gave up may not; clear
   // both (the first 256 bytes plus the 256-aligned counter block) on the caller's stream.
   const size_t groups = (size_t)B * Hkv * (size_t)((Hq / Hkv) / heads_per_cta);

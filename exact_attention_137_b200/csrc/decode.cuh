@@ -1,25 +1,34 @@
-// Single-token decode over a contiguous or paged KV cache: split-KV partials plus an
-// LSE-weighted combine pass.
+// Single-token decode over a contiguous or paged KV cache: split-KV partials merged by
+// their log-sum-exp.
 //
 // The KV cache is read once from HBM, which bounds the step (CSDN «注意力变体深挖» §一
 // and §七: decoding is memory-bound on KV reads).  Design for sm_100a:
 //
-//  * grid (split, kv head x head-subgroup, batch).  A CTA reads the K/V of one KV head
-//    for one chunk of tokens and serves the G query heads of its subgroup from that
-//    single read (GQA: the group's heads share each K/V row).
-//  * warp 4 streams the chunk through a 3-stage ring of 64-token stages with cp.async.bulk:
-//    every run of tokens that is contiguous in the cache (one page of a paged pool, or
-//    the whole stage in a dense cache) is one bulk copy.  The page ids come from the
-//    block table (gocoding §5), prefetched 32 pages ahead into the producer's lanes.
+//  * Work is counted in units of 16 tokens of one stream, a stream being the K/V of one
+//    KV head of one sequence read for a subgroup of G of its query heads (GQA: the
+//    group's heads share each K/V row, so one read serves all of them).  The streams are
+//    laid end to end, sequence-major, and a persistent grid of two CTAs per SM cuts that
+//    line into equal contiguous ranges (decode_schedule below).  Every CTA therefore
+//    reads the same number of bytes whatever the length mix, and a CTA's range is a
+//    list of segments: pieces of at most two streams shared with neighbouring CTAs, and
+//    whole streams in between.
+//  * warp 4 streams the segments through a 3-stage ring of 64-token stages with
+//    cp.async.bulk: every run of tokens that is contiguous in the cache (one page of a
+//    paged pool, or the whole stage of a dense cache) is one bulk copy, and the first
+//    stage of a segment also carries the segment's G query rows.  The page ids come
+//    from the block table (gocoding §5), prefetched 32 pages ahead into the producer's
+//    lanes.
 //  * warps 0-3 compute.  Eight lanes cover one token row (D/8 elements each, as
-//    interleaved 16-byte slices so that reads are conflict-free); per step
-//    each lane forms the partial dot products of 8 (token, head) pairs with packed fp32
-//    FMAs and a 3-level reduce-scatter across the 8 lanes leaves one complete score per
-//    lane (fewer lanes per row means less shuffle work per score).  Online softmax per
-//    head (log2 domain, ex2), then the value rows are accumulated as fp32 pairs.
-//  * each split writes its normalised partial output and its LSE; the combine kernel
-//    merges the splits of a (sequence, head) with weights exp(lse_s - LSE), the same
-//    two-way merge as the pages' online softmax, applied across splits.
+//    interleaved 16-byte slices so that reads are conflict-free); per step each lane
+//    forms the partial dot products of 8 (token, head) pairs with packed fp32 FMAs and a
+//    3-level reduce-scatter across the 8 lanes leaves one complete score per lane.
+//    Online softmax per head (log2 domain, ex2), then the value rows are accumulated as
+//    fp32 pairs.
+//  * at the end of a segment the four warps merge through the shared memory of the
+//    stage they still hold.  A whole stream writes O and LSE directly; a shared stream
+//    writes a normalised partial (O_s, lse_s) into this CTA's workspace slot, and the
+//    CTA that finishes a stream last merges all its partials with weights
+//    exp(lse_s - LSE): the pages' two-way online-softmax merge, applied across CTAs.
 #pragma once
 
 #include "common.cuh"
@@ -31,7 +40,121 @@ constexpr int kStageTokens = 64;
 constexpr int kStages = 3;
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
-constexpr int kMaxSplits = 128;  // the plan never splits a sequence into more chunks
+
+// Schedule constants.
+constexpr int kUnitTokens = 16;      // granularity of the split points
+constexpr int kMinUnitsPerCta = 8;   // fewer CTAs are used when there is less work than this each
+constexpr int kCtasPerSm = 2;        // resident CTAs per SM (registers and shared memory allow two)
+constexpr int kMaxCtas = 512;        // grid cap; sizes the workspace independently of the device
+
+// ---------------------------------------------------------------------- schedule
+//
+// Shared by the kernel and by the host-side listing (attn_decode_schedule), so both see
+// the same segments.  Y streams per sequence; sequence b has units_of(len_b) units in
+// each of its streams; the global unit line is ordered (b, y, unit).  With n CTAs over
+// `total` units, CTA i owns [begin(i), begin(i+1)), begin(i) = floor(i * total / n).
+
+__host__ __device__ __forceinline__ int units_of(int len) { return (len + kUnitTokens - 1) / kUnitTokens; }
+
+__host__ __device__ __forceinline__ int active_ctas(long long total, int launched) {
+  const long long want = (total + kMinUnitsPerCta - 1) / kMinUnitsPerCta;
+  return (int)(want < launched ? want : launched);
+}
+
+__host__ __device__ __forceinline__ long long cta_begin(int i, long long total, int n) {
+  return (long long)i * total / n;
+}
+
+// The CTA whose range holds unit x: the largest i with begin(i) <= x.
+__host__ __device__ __forceinline__ int cta_of(long long x, long long total, int n) {
+  return (int)(((x + 1) * n - 1) / total);
+}
+
+struct Segment {
+  int b, y;         // sequence, and stream within it (kv head * subgroups + subgroup)
+  int tok0, tok1;   // tokens [tok0, tok1) of the sequence
+  int slot;         // -1: the stream lies wholly in this CTA; else this CTA's partial slot (0, 1)
+  int nsplit;       // CTAs that share the stream (1 when whole)
+  long long start;  // global unit offset of the stream
+};
+
+struct Walk {
+  long long pos, hi;  // next unit of this CTA, end of its range
+  int b, y, u;        // current stream and unit offset within it
+  int len, units;     // length and units of sequence b
+  bool first;         // the next segment is this CTA's first
+};
+
+// Sequence lengths from host memory, clamped to [0, max_seqlen] (the host-side listing).
+struct HostLens {
+  const int* lens;
+  int max_seqlen;
+  __host__ __device__ int operator()(int b) const {
+    const int len = lens[b];
+    return len < 0 ? 0 : (len > max_seqlen ? max_seqlen : len);
+  }
+};
+
+// Next segment of the walk; false when the CTA's range is exhausted.  len_of(b) returns the
+// (checked) length of sequence b.
+template <class LenOf>
+__host__ __device__ __forceinline__ bool next_segment(Walk& w, const LenOf& len_of, int Y, long long total, int n,
+                                                      Segment& s) {
+  if (w.pos >= w.hi) return false;
+  while (w.u >= w.units) {  // step over finished and empty streams
+    w.u = 0;
+    if (++w.y == Y) {
+      w.y = 0;
+      ++w.b;
+      w.len = len_of(w.b);
+      w.units = units_of(w.len);
+    }
+  }
+  const long long left = w.hi - w.pos;
+  const int take = (long long)(w.units - w.u) < left ? w.units - w.u : (int)left;
+  s.b = w.b;
+  s.y = w.y;
+  s.tok0 = w.u * kUnitTokens;
+  const int t1 = (w.u + take) * kUnitTokens;
+  s.tok1 = t1 < w.len ? t1 : w.len;
+  s.start = w.pos - w.u;
+  const bool whole = w.u == 0 && take == w.units;
+  s.nsplit = whole ? 1 : cta_of(s.start + w.units - 1, total, n) - cta_of(s.start, total, n) + 1;
+  s.slot = whole ? -1 : (w.first ? 0 : 1);
+  w.pos += take;
+  w.u += take;
+  w.first = false;
+  return true;
+}
+
+// Host restatement of the start of CTA i's walk (serial scan); the kernel does the same
+// search with one warp.
+template <class LenOf>
+inline Walk walk_start_host(const LenOf& len_of, int B, int Y, long long total, int n, int i) {
+  Walk w{};
+  w.pos = cta_begin(i, total, n);
+  w.hi = cta_begin(i + 1, total, n);
+  w.first = true;
+  long long prefix = 0;
+  for (int b = 0; b < B; ++b) {
+    const int len = len_of(b);
+    const long long span = (long long)Y * units_of(len);
+    if (w.pos < prefix + span) {
+      const long long off = w.pos - prefix;
+      w.b = b;
+      w.len = len;
+      w.units = units_of(len);
+      w.y = (int)(off / w.units);
+      w.u = (int)(off - (long long)w.y * w.units);
+      return w;
+    }
+    prefix += span;
+  }
+  w.hi = w.pos;  // empty range
+  return w;
+}
+
+// ---------------------------------------------------------------------- kernel
 
 struct Params {
   const __nv_bfloat16* q;
@@ -41,25 +164,39 @@ struct Params {
   const int* block_table;  // nullptr: contiguous cache
   int block_size, max_blocks, num_blocks, max_seqlen;
   int B, Hq, Hkv;
-  int chunk, max_splits, nsub;
+  int nsub;  // query-head subgroups of G per KV head
   float scale_log2;
-  float* ws_o;    // [B, Hq, max_splits, D]
-  float* ws_lse;  // [B, Hq, max_splits]
+  float* ws_o;    // [grid][2][G][D] partial outputs per CTA slot
+  float* ws_lse;  // [grid][2][G]
   unsigned int* ws_err;
-  int* ws_cnt;    // [B, Hkv * nsub] splits finished; the last one merges and resets it
+  int* ws_cnt;    // [B][Hkv * nsub] partials finished; the last one merges and resets it
   __nv_bfloat16* o;
   float* lse;
 };
 
-template <int D>
+// The consumers' copy of the walk: consumer thread 0 advances it one segment ahead into
+// the slot the other consumers are not reading.
+struct SegSlots {
+  Walk w;
+  Segment sg[2];
+  int has[2];
+};
+
+template <int D, int G>
 struct Layout {
   static constexpr int kRow = D * 2;
   static constexpr int kStageBytes = kStageTokens * kRow;  // K (or V) bytes of one stage
-  static constexpr int kK = 0;
-  static constexpr int kV = kStages * kStageBytes;
-  static constexpr int kBar = 2 * kStages * kStageBytes;
+  static constexpr int kSlotBytes = 2 * kStageBytes;       // a stage: K rows, then V rows
+  static constexpr int kQBytes = G * kRow;                 // the segment's query rows
+  static constexpr int kQ = kStages * kSlotBytes;
+  static constexpr int kBar = kQ + kStages * kQBytes;
   static constexpr int kMisc = kBar + 2 * kStages * 8;
-  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kSeg = kMisc + 64;  // consumers' walk state and two segment slots
+  static constexpr int kBytes = kSeg + 128;
+  // The end-of-segment merge and the cross-CTA merge run in the held stage's memory.
+  static_assert(4 * (2 * kConsumerWarps * G + kConsumerWarps * G * D) <= kSlotBytes, "warp merge fits a stage");
+  static_assert(4 * G * kMaxCtas <= kSlotBytes, "merge weights fit a stage");
+  static_assert(sizeof(SegSlots) <= kBytes - kSeg, "segment slots fit");
 };
 
 __device__ __forceinline__ void flag_error(const Params& p, unsigned int f) {
@@ -79,23 +216,75 @@ __device__ __forceinline__ int checked_len(const Params& p, int b, bool report) 
   return len;
 }
 
-__device__ __forceinline__ void unpack8(uint4 w, float (&f)[8]) {
-  f[0] = bf16lo(w.x);
-  f[1] = bf16hi(w.x);
-  f[2] = bf16lo(w.y);
-  f[3] = bf16hi(w.y);
-  f[4] = bf16lo(w.z);
-  f[5] = bf16hi(w.z);
-  f[6] = bf16lo(w.w);
-  f[7] = bf16hi(w.w);
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(addr));
   return v;
+}
+
+__device__ __forceinline__ long long shfl_ll(long long v, int src) {
+  const int lo = __shfl_sync(0xffffffffu, (int)(v & 0xffffffffll), src);
+  const int hi = __shfl_sync(0xffffffffu, (int)(v >> 32), src);
+  return ((long long)hi << 32) | (unsigned int)lo;
+}
+
+__device__ __forceinline__ long long shfl_up_ll(long long v, int d) {
+  const int lo = __shfl_up_sync(0xffffffffu, (int)(v & 0xffffffffll), d);
+  const int hi = __shfl_up_sync(0xffffffffu, (int)(v >> 32), d);
+  return ((long long)hi << 32) | (unsigned int)lo;
+}
+
+// Units over all streams; every lane of the warp returns the same value.
+__device__ __forceinline__ long long total_units(const Params& p, int Y, int lane, bool report) {
+  long long sum = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    sum += b < p.B ? units_of(checked_len(p, b, report)) : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += shfl_ll(sum, lane ^ o);
+  return sum * Y;
+}
+
+// walk_start_host with a warp: a prefix scan over the sequences, 32 at a time.
+__device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long total, int n, int i, int lane) {
+  Walk w;
+  w.pos = cta_begin(i, total, n);
+  w.hi = cta_begin(i + 1, total, n);
+  w.first = true;
+  w.b = 0;
+  w.y = 0;
+  w.u = 0;
+  w.len = 0;
+  w.units = 0;
+  long long prefix = 0;
+  for (int b0 = 0; b0 < p.B; b0 += 32) {
+    const int b = b0 + lane;
+    const int len = b < p.B ? checked_len(p, b, false) : 0;
+    const long long span = (long long)Y * units_of(len);
+    long long incl = span;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const long long t = shfl_up_ll(incl, d);
+      if (lane >= d) incl += t;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, w.pos < prefix + incl);
+    if (hit) {
+      const int l = __ffs(hit) - 1;
+      const long long off = w.pos - (prefix + shfl_ll(incl - span, l));
+      w.b = b0 + l;
+      w.len = __shfl_sync(0xffffffffu, len, l);
+      w.units = units_of(w.len);
+      w.y = (int)(off / w.units);
+      w.u = (int)(off - (long long)w.y * w.units);
+      return w;
+    }
+    prefix += shfl_ll(incl, 31);
+  }
+  w.hi = w.pos;
+  return w;
 }
 
 // Recursive-halving reduce-scatter over the LPT lanes of a group: on return lane j of
@@ -115,8 +304,14 @@ __device__ __forceinline__ float reduce_scatter(float (&vals)[LPT], int j) {
   return vals[0];
 }
 
+// Named barrier 1 over the consumer warps (the producer never takes part).
+template <int kCount>
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory");
+}
+
 template <int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   // Lanes per token row: 8, except D=128 with 8 heads per CTA, where 16 lanes halve the
   // per-lane query and accumulator registers.
   constexpr int LPT = (D == 128 && G == 8) ? 16 : 8;
@@ -126,40 +321,39 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params 
   constexpr int GPW = 32 / LPT;    // lane groups per warp
   constexpr int TPW = GPW * TOK;   // tokens per warp step (= 32 / G)
   constexpr int UNITS = kStageTokens / TPW;  // warp steps per stage (= G)
+  constexpr int kCon = kConsumerWarps * 32;
   static_assert(G <= LPT && TOK * G == LPT, "heads per CTA must divide the lanes per token");
   static_assert(EPL % 8 == 0, "each lane reads whole 16-byte slices");
-  constexpr bool kJoint = true;
-  using L = Layout<D>;
+  using L = Layout<D, G>;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
   auto full_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * s; };
   auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (kStages + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
-
-  const int b = blockIdx.z;
-  const int split = blockIdx.x;
-  const int len = checked_len(p, b, split == 0 && blockIdx.y == 0 && threadIdx.x == 0);
-  const int nsplit = (len + p.chunk - 1) / p.chunk;
-  const int kvh0 = blockIdx.y / p.nsub;
-  const int hbase = kvh0 * (p.Hq / p.Hkv) + (blockIdx.y - kvh0 * p.nsub) * G;
-  if (nsplit == 0 && split == 0) {  // empty sequence: O = 0, LSE = -inf
-    for (int idx = threadIdx.x; idx < G * D; idx += blockDim.x) {
-      const int hh = idx / D, d = idx - hh * D;
-      p.o[((size_t)b * p.Hq + hbase + hh) * D + d] = __float2bfloat16_rn(0.f);
-      if (p.lse != nullptr && d == 0) p.lse[(size_t)b * p.Hq + hbase + hh] = -INFINITY;
-    }
-  }
-  if (split >= nsplit) return;
-  const int t0 = split * p.chunk;
-  const int t1 = min(len, t0 + p.chunk);
-  const int niters = (t1 - t0 + kStageTokens - 1) / kStageTokens;
-  const int kvh = blockIdx.y / p.nsub;
-  const int sub = blockIdx.y - kvh * p.nsub;
-  const int g = p.Hq / p.Hkv;
-  const int h0 = kvh * g + sub * G;
+  volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  float* lse_f = reinterpret_cast<float*>(smem + L::kMisc + 32);  // [G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Y = p.Hkv * p.nsub;
+  const int g = p.Hq / p.Hkv;
+  const long long total = total_units(p, Y, lane, blockIdx.x == 0 && warp == 0);
+
+  // Empty sequences have no units; CTA i writes O = 0, LSE = -inf for b = i mod grid.
+  if (warp < kConsumerWarps) {
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+      if (checked_len(p, b, false) != 0) continue;
+      for (int idx = threadIdx.x; idx < p.Hq * D; idx += kCon) {
+        p.o[(size_t)b * p.Hq * D + idx] = __float2bfloat16_rn(0.f);
+        if (p.lse != nullptr && idx % D == 0) p.lse[(size_t)b * p.Hq + idx / D] = -INFINITY;
+      }
+    }
+  }
+  const int n = active_ctas(total, gridDim.x);
+  if ((int)blockIdx.x >= n) return;
+  auto len_of = [&](int b) -> int { return checked_len(p, b, false); };
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(full_bar(s), 1);
@@ -169,59 +363,71 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params 
     fence_barrier_init();
   }
   __syncthreads();
+  Walk w = walk_start(p, Y, total, n, blockIdx.x, lane);
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ bulk-copy producer
     const int bs = p.block_size;
     const bool paged = p.block_table != nullptr;
-    const int* table = paged ? p.block_table + (size_t)b * p.max_blocks : nullptr;
-    auto load_id = [&](int page) -> int {
-      return (paged && page < p.max_blocks) ? __ldg(table + page) : -1;
-    };
-    int cur_first = t0 / bs;
-    int nxt_first = cur_first + 32;
-    int cur_id = load_id(cur_first + lane);
-    int nxt_id = load_id(nxt_first + lane);
     int last_fill[kStages];
     for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
-    for (int it = 0; it < niters; ++it) {
-      const int s = it % kStages;
-      const int f = it / kStages;
-      if (f > 0) {
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), (f - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-      const int a = t0 + it * kStageTokens;
-      const int e = min(t1, a + kStageTokens);
-      const uint32_t dk = sbase + L::kK + s * L::kStageBytes;
-      const uint32_t dv = sbase + L::kV + s * L::kStageBytes;
-      for (int tok = a; tok < e;) {
-        const int page = tok / bs;
-        const int slot = tok - page * bs;
-        const int run = min(bs - slot, e - tok);
-        while (page >= cur_first + 32) {
-          cur_id = nxt_id;
-          cur_first = nxt_first;
-          nxt_first += 32;
-          nxt_id = load_id(nxt_first + lane);
+    int it = 0;
+    bool alive = true;
+    Segment sg;
+    while (alive && next_segment(w, len_of, Y, total, n, sg)) {
+      const int kvh = sg.y / p.nsub;
+      const int h0 = kvh * g + (sg.y - kvh * p.nsub) * G;
+      const int* table = paged ? p.block_table + (size_t)sg.b * p.max_blocks : nullptr;
+      auto load_id = [&](int page) -> int {
+        return (paged && page < p.max_blocks) ? __ldg(table + page) : -1;
+      };
+      int cur_first = sg.tok0 / bs;
+      int nxt_first = cur_first + 32;
+      int cur_id = load_id(cur_first + lane);
+      int nxt_id = load_id(nxt_first + lane);
+      for (int a = sg.tok0; a < sg.tok1; a += kStageTokens, ++it) {
+        const int s = it % kStages;
+        const int f = it / kStages;
+        if (f > 0) {
+          alive = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), (f - 1) & 1, abort_flag));
+          if (!alive) break;
         }
-        const int blk = paged ? __shfl_sync(0xffffffffu, cur_id, page - cur_first) : b;
-        if (lane == 0) {
-          if (blk < 0 || blk >= p.num_blocks) {
-            flag_error(p, ATTN_DEV_BAD_BLOCK);
-          } else {
-            const size_t off = (((size_t)blk * p.Hkv + kvh) * (size_t)bs + slot) * D;
-            const uint32_t bytes = (uint32_t)run * L::kRow;
-            const uint32_t dst = (uint32_t)(tok - a) * L::kRow;
-            mbar_expect_tx(full_bar(s), 2u * bytes);
-            bulk_load(dk + dst, p.kc + off, bytes, full_bar(s));
-            bulk_load(dv + dst, p.vc + off, bytes, full_bar(s));
+        const int e = min(sg.tok1, a + kStageTokens);
+        const uint32_t dk = sbase + s * L::kSlotBytes;
+        const uint32_t dv = dk + L::kStageBytes;
+        if (a == sg.tok0 && lane == 0) {
+          mbar_expect_tx(full_bar(s), (uint32_t)L::kQBytes);
+          bulk_load(sbase + L::kQ + s * L::kQBytes, p.q + ((size_t)sg.b * p.Hq + h0) * D, (uint32_t)L::kQBytes,
+                    full_bar(s));
+        }
+        for (int tok = a; tok < e;) {
+          const int page = tok / bs;
+          const int slot = tok - page * bs;
+          const int run = min(bs - slot, e - tok);
+          while (page >= cur_first + 32) {
+            cur_id = nxt_id;
+            cur_first = nxt_first;
+            nxt_first += 32;
+            nxt_id = load_id(nxt_first + lane);
           }
+          const int blk = paged ? __shfl_sync(0xffffffffu, cur_id, page - cur_first) : sg.b;
+          if (lane == 0) {
+            if (blk < 0 || blk >= p.num_blocks) {
+              flag_error(p, ATTN_DEV_BAD_BLOCK);
+            } else {
+              const size_t off = (((size_t)blk * p.Hkv + kvh) * (size_t)bs + slot) * D;
+              const uint32_t bytes = (uint32_t)run * L::kRow;
+              const uint32_t dst = (uint32_t)(tok - a) * L::kRow;
+              mbar_expect_tx(full_bar(s), 2u * bytes);
+              bulk_load(dk + dst, p.kc + off, bytes, full_bar(s));
+              bulk_load(dv + dst, p.vc + off, bytes, full_bar(s));
+            }
+          }
+          tok += run;
         }
-        tok += run;
+        if (lane == 0) mbar_arrive(full_bar(s));
+        last_fill[s] = f;
       }
-      if (lane == 0) mbar_arrive(full_bar(s));
-      last_fill[s] = f;
     }
     if (*abort_flag && lane == 0) {
       // Consumers gave up: let copies already in flight land before the CTA exits.
@@ -233,245 +439,281 @@ __global__ void __launch_bounds__(kThreads, 2) decode_split_kernel(const Params 
   }
 
   // -------------------------------------------------------------- consumers
-  // Lane j of lane group gi owns the 16-byte slices j, j + 8, ... (8 elements each) of every
-  // token row, so the 8 lanes of a group read 128 contiguous bytes per access (no bank
-  // conflicts); a group covers one row, so a score is complete after a 3-level
-  // reduce-scatter.
+  // Lane j of lane group gi owns the 16-byte slices j, j + LPT, ... of every token row, so
+  // the LPT lanes of a group read contiguous bytes per access (no bank conflicts); a group
+  // covers one row, so a score is complete after the reduce-scatter.
   const int gi = lane / LPT;
   const int j = lane - gi * LPT;
-  uint64_t q2[G][WPL];  // this lane's query elements per head, as fp32 pairs
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)b * p.Hq + h0 + hh) * D) + j;
-#pragma unroll
-    for (int v4 = 0; v4 < EPL / 8; ++v4) {
-      const uint4 w = __ldg(src + LPT * v4);
-      q2[hh][4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
-      q2[hh][4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
-      q2[hh][4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
-      q2[hh][4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
-    }
-  }
   const float c = p.scale_log2;
-  float m_own = -INFINITY, l_own = 0.f;
-  uint64_t acc[G][WPL];
+  SegSlots* ss = reinterpret_cast<SegSlots*>(smem + L::kSeg);
+  volatile int* has = ss->has;
+  if (threadIdx.x == 0) {
+    has[0] = next_segment(w, len_of, Y, total, n, ss->sg[0]);
+    ss->w = w;
+  }
+  consumer_sync<kCon>();
+  int it = 0;
+  for (int k = 0; has[k & 1]; ++k) {
+    if (threadIdx.x == 0) {  // one segment ahead, into the other slot
+      Walk wn = ss->w;
+      has[(k + 1) & 1] = next_segment(wn, len_of, Y, total, n, ss->sg[(k + 1) & 1]);
+      ss->w = wn;
+    }
+    const Segment& sg = ss->sg[k & 1];
+    const int kvh = sg.y / p.nsub;
+    const int h0 = kvh * g + (sg.y - kvh * p.nsub) * G;
+    const int nst = (sg.tok1 - sg.tok0 + kStageTokens - 1) / kStageTokens;
+    uint64_t q2[G][WPL];  // this lane's query elements per head, as fp32 pairs
+    float m_own = -INFINITY, l_own = 0.f;
+    uint64_t acc[G][WPL];
 #pragma unroll
-  for (int hh = 0; hh < G; ++hh)
+    for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-    for (int e = 0; e < WPL; ++e) acc[hh][e] = 0ull;
+      for (int e = 0; e < WPL; ++e) acc[hh][e] = 0ull;
 
-  bool ok = true;
-  for (int it = 0; it < niters; ++it) {
-    const int s = it % kStages;
-    ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / kStages) & 1, abort_flag));
-    if (!ok) break;
-    const int nv = min(kStageTokens, t1 - (t0 + it * kStageTokens));
-    const uint32_t sk = sbase + L::kK + s * L::kStageBytes;
-    const uint32_t sv = sbase + L::kV + s * L::kStageBytes;
-    // Each warp takes two units of the stage at a time (u and u + 4 warps): their dot
-    // products and reductions are independent, which gives the warp twice the ILP; they
-    // share one max update and one rescale.  A second unit past the stage is empty.
-    for (int u = warp; u < UNITS; u += (kJoint ? 2 : 1) * kConsumerWarps) {
-      const int u1 = u + kConsumerWarps;
-      const bool has1 = kJoint && u1 < UNITS;
-      const int tb0 = u * TPW + gi * TOK;                   // first token of this lane group
-      const int tb1 = (has1 ? u1 : u) * TPW + gi * TOK;
-      float vals0[LPT], vals1[LPT];
+    bool ok = true;
+    int held = 0;
+    for (int st = 0; st < nst; ++st) {
+      const int s = it % kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / kStages) & 1, abort_flag));
+      if (!ok) break;
+      ++it;
+      held = s;
+      if (st == 0) {
+        const uint32_t sq = sbase + L::kQ + s * L::kQBytes;
 #pragma unroll
-      for (int tt = 0; tt < TOK; ++tt) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          uint64_t k2[WPL];
+        for (int hh = 0; hh < G; ++hh)
 #pragma unroll
           for (int v4 = 0; v4 < EPL / 8; ++v4) {
-            const uint4 w = lds128(sk + (uint32_t)((x ? tb1 : tb0) + tt) * L::kRow + 16u * (j + LPT * v4));
-            k2[4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
-            k2[4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
-            k2[4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
-            k2[4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+            const uint4 wq = lds128(sq + hh * L::kRow + 16u * (j + LPT * v4));
+            q2[hh][4 * v4 + 0] = f2pack(bf16lo(wq.x), bf16hi(wq.x));
+            q2[hh][4 * v4 + 1] = f2pack(bf16lo(wq.y), bf16hi(wq.y));
+            q2[hh][4 * v4 + 2] = f2pack(bf16lo(wq.z), bf16hi(wq.z));
+            q2[hh][4 * v4 + 3] = f2pack(bf16lo(wq.w), bf16hi(wq.w));
           }
+      }
+      const int nv = min(kStageTokens, sg.tok1 - (sg.tok0 + st * kStageTokens));
+      const uint32_t sk = sbase + s * L::kSlotBytes;
+      const uint32_t sv = sk + L::kStageBytes;
+      // Each warp takes two units of the stage at a time (u and u + 4 warps): their dot
+      // products and reductions are independent, which gives the warp twice the ILP; they
+      // share one max update and one rescale.  A second unit past the stage is empty.
+      for (int u = warp; u < UNITS; u += 2 * kConsumerWarps) {
+        const int u1 = u + kConsumerWarps;
+        const bool has1 = u1 < UNITS;
+        const int tb0 = u * TPW + gi * TOK;  // first token of this lane group
+        const int tb1 = (has1 ? u1 : u) * TPW + gi * TOK;
+        float vals0[LPT], vals1[LPT];
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            uint64_t d2 = fmul2(q2[hh][0], k2[0]);
+        for (int tt = 0; tt < TOK; ++tt) {
 #pragma unroll
-            for (int e = 1; e < WPL; ++e) d2 = ffma2(q2[hh][e], k2[e], d2);
-            float lo, hi;
-            f2unpack(d2, lo, hi);
-            if (x) vals1[tt * G + hh] = lo + hi;
-            else vals0[tt * G + hh] = lo + hi;
+          for (int x = 0; x < 2; ++x) {
+            uint64_t k2[WPL];
+#pragma unroll
+            for (int v4 = 0; v4 < EPL / 8; ++v4) {
+              const uint4 wk = lds128(sk + (uint32_t)((x ? tb1 : tb0) + tt) * L::kRow + 16u * (j + LPT * v4));
+              k2[4 * v4 + 0] = f2pack(bf16lo(wk.x), bf16hi(wk.x));
+              k2[4 * v4 + 1] = f2pack(bf16lo(wk.y), bf16hi(wk.y));
+              k2[4 * v4 + 2] = f2pack(bf16lo(wk.z), bf16hi(wk.z));
+              k2[4 * v4 + 3] = f2pack(bf16lo(wk.w), bf16hi(wk.w));
+            }
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+              uint64_t d2 = fmul2(q2[hh][0], k2[0]);
+#pragma unroll
+              for (int e = 1; e < WPL; ++e) d2 = ffma2(q2[hh][e], k2[e], d2);
+              float lo, hi;
+              f2unpack(d2, lo, hi);
+              if (x) vals1[tt * G + hh] = lo + hi;
+              else vals0[tt * G + hh] = lo + hi;
+            }
           }
         }
-      }
-      const float score0 = reduce_scatter<LPT>(vals0, j);
-      const float score1 = reduce_scatter<LPT>(vals1, j);
-      const float x0 = (tb0 + j / G < nv) ? score0 * c : -INFINITY;
-      const float x1 = (has1 && tb1 + j / G < nv) ? score1 * c : -INFINITY;
-      float mx = fmaxf(x0, x1);
+        const float score0 = reduce_scatter<LPT>(vals0, j);
+        const float score1 = reduce_scatter<LPT>(vals1, j);
+        const float x0 = (tb0 + j / G < nv) ? score0 * c : -INFINITY;
+        const float x1 = (has1 && tb1 + j / G < nv) ? score1 * c : -INFINITY;
+        float mx = fmaxf(x0, x1);
 #pragma unroll
-      for (int o = G; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_new = fmaxf(m_own, mx);
-      const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_own - m_new);
-      const float mu = (m_new == -INFINITY) ? 0.f : m_new;
-      const float pr0 = fast_exp2(x0 - mu), pr1 = fast_exp2(x1 - mu);
-      l_own = l_own * alpha + (pr0 + pr1);
-      m_own = m_new;
-      if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const float ah = __shfl_sync(0xffffffffu, alpha, hh);
-          const uint64_t a2 = f2pack(ah, ah);
-#pragma unroll
-          for (int e = 0; e < WPL; ++e) acc[hh][e] = fmul2(acc[hh][e], a2);
-        }
-      }
-#pragma unroll
-      for (int tt = 0; tt < TOK; ++tt) {
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          uint64_t v2[WPL];
-          const int tok = (x ? tb1 : tb0) + tt;
-#pragma unroll
-          for (int v4 = 0; v4 < EPL / 8; ++v4) {
-            const uint4 w = lds128(sv + (uint32_t)tok * L::kRow + 16u * (j + LPT * v4));
-            v2[4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
-            v2[4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
-            v2[4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
-            v2[4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
-          }
-          const bool tv = (x == 0 || has1) && tok < nv;
+        for (int o = G; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float m_new = fmaxf(m_own, mx);
+        const float alpha = (m_new == -INFINITY) ? 1.f : fast_exp2(m_own - m_new);
+        const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+        const float pr0 = fast_exp2(x0 - mu), pr1 = fast_exp2(x1 - mu);
+        l_own = l_own * alpha + (pr0 + pr1);
+        m_own = m_new;
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) {
-            const float ph = __shfl_sync(0xffffffffu, x ? pr1 : pr0, gi * LPT + tt * G + hh);
-            if (tv) {
-              const uint64_t p2 = f2pack(ph, ph);
+            const float ah = __shfl_sync(0xffffffffu, alpha, hh);
+            const uint64_t a2 = f2pack(ah, ah);
 #pragma unroll
-              for (int e = 0; e < WPL; ++e) acc[hh][e] = ffma2(p2, v2[e], acc[hh][e]);
+            for (int e = 0; e < WPL; ++e) acc[hh][e] = fmul2(acc[hh][e], a2);
+          }
+        }
+#pragma unroll
+        for (int tt = 0; tt < TOK; ++tt) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            uint64_t v2[WPL];
+            const int tok = (x ? tb1 : tb0) + tt;
+#pragma unroll
+            for (int v4 = 0; v4 < EPL / 8; ++v4) {
+              const uint4 wv = lds128(sv + (uint32_t)tok * L::kRow + 16u * (j + LPT * v4));
+              v2[4 * v4 + 0] = f2pack(bf16lo(wv.x), bf16hi(wv.x));
+              v2[4 * v4 + 1] = f2pack(bf16lo(wv.y), bf16hi(wv.y));
+              v2[4 * v4 + 2] = f2pack(bf16lo(wv.z), bf16hi(wv.z));
+              v2[4 * v4 + 3] = f2pack(bf16lo(wv.w), bf16hi(wv.w));
+            }
+            const bool tv = (x == 0 || has1) && tok < nv;
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) {
+              const float ph = __shfl_sync(0xffffffffu, x ? pr1 : pr0, gi * LPT + tt * G + hh);
+              if (tv) {
+                const uint64_t p2 = f2pack(ph, ph);
+#pragma unroll
+                for (int e = 0; e < WPL; ++e) acc[hh][e] = ffma2(p2, v2[e], acc[hh][e]);
+              }
             }
           }
         }
       }
+      if (st + 1 < nst) {  // the segment's last stage stays held for the merge below
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+      }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty_bar(s));
-  }
 
-  // Merge lane groups of this warp: per head, acc summed over groups, l over all lanes.
-  float accf[G][EPL];
-#pragma unroll
-  for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-    for (int e = 0; e < WPL; ++e) f2unpack(acc[hh][e], accf[hh][2 * e], accf[hh][2 * e + 1]);
-#pragma unroll
-  for (int o = LPT; o < 32; o <<= 1)
+    // ------------------------------------------------ end of segment: merge the warps
+    // Lane groups of this warp first: per head, acc summed over groups, l over all lanes.
+    float accf[G][EPL];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) accf[hh][e] += __shfl_xor_sync(0xffffffffu, accf[hh][e], o);
-  float l_sum = l_own;
+      for (int e = 0; e < WPL; ++e) f2unpack(acc[hh][e], accf[hh][2 * e], accf[hh][2 * e + 1]);
 #pragma unroll
-  for (int o = G; o < 32; o <<= 1) l_sum += __shfl_xor_sync(0xffffffffu, l_sum, o);
-
-  // Merge the consumer warps through shared memory (the ring is idle now).
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  float* m_s = reinterpret_cast<float*>(smem);                 // [warps][G]
-  float* l_s = m_s + kConsumerWarps * G;                       // [warps][G]
-  float* a_s = l_s + kConsumerWarps * G;                       // [warps][G][D]
-  // Outside the ring: in-flight copies of an aborted call must not touch these.
-  volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  // Any consumer that gave up set *abort_flag; snapshot it between two barriers so that
-  // every consumer warp takes the same branch below (named barriers never time out).
-  if (threadIdx.x == 0) *ok_s = (*abort_flag == 0);
-  if (ok) {
-    if (lane < G) {
-      m_s[warp * G + lane] = m_own;  // lane hh holds head hh
-      l_s[warp * G + lane] = l_sum;
-    }
-    if (gi == 0) {
+    for (int o = LPT; o < 32; o <<= 1)
 #pragma unroll
       for (int hh = 0; hh < G; ++hh)
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) a_s[(warp * G + hh) * D + 8 * (j + LPT * (e >> 3)) + (e & 7)] = accf[hh][e];
-    }
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  if (!*ok_s) return;
-  const size_t bh0 = (size_t)b * p.Hq + h0;
-  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
-    const int hh = idx / D, d = idx - hh * D;
-    float M = -INFINITY;
+        for (int e = 0; e < EPL; ++e) accf[hh][e] += __shfl_xor_sync(0xffffffffu, accf[hh][e], o);
+    float l_sum = l_own;
 #pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, m_s[w * G + hh]);
-    float Lsum = 0.f, O = 0.f;
-    if (M != -INFINITY) {
+    for (int o = G; o < 32; o <<= 1) l_sum += __shfl_xor_sync(0xffffffffu, l_sum, o);
+
+    // Then the consumer warps, in the held stage's memory (every copy into it has landed
+    // and the producer cannot refill it until the empty arrivals at the end).
+    consumer_sync<kCon>();
+    float* m_s = reinterpret_cast<float*>(smem + held * L::kSlotBytes);  // [warps][G]
+    float* l_s = m_s + kConsumerWarps * G;                                // [warps][G]
+    float* a_s = l_s + kConsumerWarps * G;                                // [warps][G][D]
+    // Any consumer that gave up set *abort_flag; snapshot it between two barriers so that
+    // every consumer warp takes the same branch below (named barriers never time out).
+    if (threadIdx.x == 0) *ok_s = (*abort_flag == 0);
+    if (ok) {
+      if (lane < G) {
+        m_s[warp * G + lane] = m_own;  // lane hh holds head hh
+        l_s[warp * G + lane] = l_sum;
+      }
+      if (gi == 0) {
 #pragma unroll
-      for (int w = 0; w < kConsumerWarps; ++w) {
-        const float sc = fast_exp2(m_s[w * G + hh] - M);
-        Lsum += l_s[w * G + hh] * sc;
-        O += a_s[(w * G + hh) * D + d] * sc;
+        for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+          for (int e = 0; e < EPL; ++e)
+            a_s[(warp * G + hh) * D + 8 * (j + LPT * (e >> 3)) + (e & 7)] = accf[hh][e];
       }
     }
-    const float o_val = Lsum > 0.f ? O / Lsum : 0.f;
-    const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
-    if (nsplit == 1) {  // the only split: write the result directly
-      p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);
-      if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_val;
-    } else {
-      const size_t slot = (bh0 + hh) * p.max_splits + split;
-      p.ws_o[slot * D + d] = o_val;
-      if (d == 0) p.ws_lse[slot] = lse_val;
+    consumer_sync<kCon>();
+    if (!*ok_s) return;
+    const size_t bh0 = (size_t)sg.b * p.Hq + h0;
+    const size_t row = (size_t)blockIdx.x * 2 + (sg.slot > 0 ? 1 : 0);
+    for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
+      const int hh = idx / D, d = idx - hh * D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w4 = 0; w4 < kConsumerWarps; ++w4) M = fmaxf(M, m_s[w4 * G + hh]);
+      float Lsum = 0.f, O = 0.f;
+      if (M != -INFINITY) {
+#pragma unroll
+        for (int w4 = 0; w4 < kConsumerWarps; ++w4) {
+          const float sc = fast_exp2(m_s[w4 * G + hh] - M);
+          Lsum += l_s[w4 * G + hh] * sc;
+          O += a_s[(w4 * G + hh) * D + d] * sc;
+        }
+      }
+      const float o_val = Lsum > 0.f ? O / Lsum : 0.f;
+      const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+      if (sg.slot < 0) {  // the whole stream: write the result directly
+        p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);
+        if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_val;
+      } else {
+        p.ws_o[(row * G + hh) * D + d] = o_val;
+        if (d == 0) p.ws_lse[row * G + hh] = lse_val;
+      }
     }
-  }
-  if (nsplit == 1) return;
 
-  // The last split of this (sequence, head group) to finish merges all partials.
-  __threadfence();
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  int* cnt = p.ws_cnt + (size_t)b * gridDim.y + blockIdx.y;
-  if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == nsplit - 1);
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  if (!*last_s) return;
-  __threadfence();
-  // Stage the partial LSEs in shared memory (one independent load per thread), turn them
-  // into merge weights exp(lse_s - LSE), then combine the partial outputs.
-  float* w_s = reinterpret_cast<float*>(smem);  // [G][max_splits]
-  float* lse_f = w_s + G * kMaxSplits;          // [G]
-  for (int idx = threadIdx.x; idx < G * nsplit; idx += kConsumerWarps * 32) {
-    const int hh = idx / nsplit, sp = idx - hh * nsplit;
-    w_s[hh * kMaxSplits + sp] = __ldcg(p.ws_lse + (bh0 + hh) * p.max_splits + sp);
-  }
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  if (threadIdx.x < G) {
-    float* w = w_s + threadIdx.x * kMaxSplits;
-    float M = -INFINITY;
-    for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, w[sp]);
-    float lse = -INFINITY;
-    if (M != -INFINITY) {
-      float Lsum = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) Lsum += expf(w[sp] - M);
-      lse = M + logf(Lsum);
+    if (sg.slot >= 0) {
+      // The last CTA of this stream to finish merges all its partials.
+      __threadfence();
+      consumer_sync<kCon>();
+      int* cnt = p.ws_cnt + (size_t)sg.b * Y + sg.y;
+      if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == sg.nsplit - 1);
+      consumer_sync<kCon>();
+      if (*last_s) {
+        __threadfence();
+        // Partial k of the stream is CTA i0 + k's; only the first of those CTAs can hold the
+        // stream in its second slot (when its range starts before the stream).
+        const int i0 = cta_of(sg.start, total, n);
+        const int slot0 = cta_begin(i0, total, n) >= sg.start ? 0 : 1;
+        const int ns = sg.nsplit;
+        float* w_s = reinterpret_cast<float*>(smem + held * L::kSlotBytes);  // [G][kMaxCtas]
+        for (int idx = threadIdx.x; idx < G * ns; idx += kCon) {
+          const int hh = idx / ns, k = idx - hh * ns;
+          const size_t r = (size_t)(i0 + k) * 2 + (k == 0 ? slot0 : 0);
+          w_s[hh * kMaxCtas + k] = __ldcg(p.ws_lse + r * G + hh);
+        }
+        consumer_sync<kCon>();
+        if (threadIdx.x < G) {
+          float* wh = w_s + threadIdx.x * kMaxCtas;
+          float M = -INFINITY;
+          for (int k = 0; k < ns; ++k) M = fmaxf(M, wh[k]);
+          float lse = -INFINITY;
+          if (M != -INFINITY) {
+            float Lsum = 0.f;
+            for (int k = 0; k < ns; ++k) Lsum += expf(wh[k] - M);
+            lse = M + logf(Lsum);
+          }
+          for (int k = 0; k < ns; ++k) wh[k] = lse == -INFINITY ? 0.f : expf(wh[k] - lse);
+          lse_f[threadIdx.x] = lse;
+        }
+        consumer_sync<kCon>();
+        const size_t rstride = (size_t)2 * G * D;  // consecutive CTAs' partials
+        const size_t r0 = (size_t)i0 * 2 + slot0;
+        for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
+          const int hh = idx / D, d = idx - hh * D;
+          const float* wh = w_s + hh * kMaxCtas;
+          // partial 0 sits in row r0; partial k >= 1 in row 2 * (i0 + k)
+          float out0 = wh[0] * __ldcg(p.ws_o + (r0 * G + hh) * D + d);
+          float out1 = 0.f, out2 = 0.f, out3 = 0.f;
+          const float* o_s = p.ws_o + ((size_t)i0 * 2 * G + hh) * D + d;
+          int k = 1;
+          for (; k + 3 <= ns; k += 3) {
+            out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
+            out2 = fmaf(wh[k + 1], __ldcg(o_s + (k + 1) * rstride), out2);
+            out3 = fmaf(wh[k + 2], __ldcg(o_s + (k + 2) * rstride), out3);
+          }
+          for (; k < ns; ++k) out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
+          p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
+          if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
+        }
+        if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
+      }
     }
-    for (int sp = 0; sp < nsplit; ++sp) w[sp] = lse == -INFINITY ? 0.f : expf(w[sp] - lse);
-    lse_f[threadIdx.x] = lse;
+    // Release the held stage once every consumer is done with its memory.
+    consumer_sync<kCon>();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty_bar(held));
   }
-  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32));
-  for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
-    const int hh = idx / D, d = idx - hh * D;
-    const float* w = w_s + hh * kMaxSplits;
-    const float* o_s = p.ws_o + (bh0 + hh) * p.max_splits * D + d;
-    float out0 = 0.f, out1 = 0.f, out2 = 0.f, out3 = 0.f;
-    int sp = 0;
-    for (; sp + 4 <= nsplit; sp += 4) {
-      out0 = fmaf(w[sp], __ldcg(o_s + (size_t)sp * D), out0);
-      out1 = fmaf(w[sp + 1], __ldcg(o_s + (size_t)(sp + 1) * D), out1);
-      out2 = fmaf(w[sp + 2], __ldcg(o_s + (size_t)(sp + 2) * D), out2);
-      out3 = fmaf(w[sp + 3], __ldcg(o_s + (size_t)(sp + 3) * D), out3);
-    }
-    for (; sp < nsplit; ++sp) out0 = fmaf(w[sp], __ldcg(o_s + (size_t)sp * D), out0);
-    p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
-    if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
-  }
-  if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
 }
 
 }  // namespace dec

@@ -37,13 +37,14 @@ def torch_dtype(name: str) -> torch.dtype:
 
 
 def _randn(shape, gen: torch.Generator, dtype: torch.dtype, chunk_elems: int = 1 << 26) -> torch.Tensor:
-    """N(0,1) fp32 draws rounded to ``dtype``, produced in chunks to bound host memory."""
-    out = torch.empty(shape, dtype=dtype)
+    """N(0,1) fp32 draws rounded to ``dtype``, produced in chunks to bound memory, on the
+    generator's device."""
+    out = torch.empty(shape, dtype=dtype, device=gen.device)
     flat = out.view(-1)
     n = flat.numel()
     for s in range(0, n, chunk_elems):
         e = min(n, s + chunk_elems)
-        flat[s:e] = torch.randn(e - s, generator=gen, dtype=torch.float32).to(dtype)
+        flat[s:e] = torch.randn(e - s, generator=gen, dtype=torch.float32, device=gen.device).to(dtype)
     return out
 
 
@@ -102,13 +103,17 @@ def decode_contiguous_inputs(B: int, Hq: int, Hkv: int, D: int, cap: int, len_lo
 
 
 def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_lo: int, len_hi: int,
-                        seed: int = 0, max_blocks: int | None = None, seqlens=None, extra_blocks: int = 0):
+                        seed: int = 0, max_blocks: int | None = None, seqlens=None, extra_blocks: int = 0,
+                        device=None):
     """One query token per sequence and a paged pool ``[num_blocks,Hkv,block_size,D]`` (bf16).
 
     The pool has ``sum(ceil(len/block_size)) + extra_blocks`` blocks; a seeded
     permutation of the pool assigns physical blocks to the sequences' logical blocks
     in order.  ``block_table`` is int32 ``[B, max_blocks]`` padded with -1.  Slots
     past a sequence's last token, and every slot of unassigned blocks, hold NaN.
+
+    ``device`` (timing-only inputs): draw q and the pool with a generator on that device,
+    seeded the same way, instead of on the CPU; lengths and the table are unchanged.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     lens = _lengths(rng, B, len_lo, len_hi) if seqlens is None else np.asarray(seqlens, dtype=np.int32)
@@ -123,7 +128,7 @@ def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_
     for b in range(B):
         table[b, : nblk[b]] = perm[off : off + nblk[b]]
         off += int(nblk[b])
-    gen = torch.Generator("cpu").manual_seed(seed)
+    gen = torch.Generator("cpu" if device is None else device).manual_seed(seed)
     q = _randn((B, Hq, D), gen, torch.bfloat16)
     k = _randn((total, Hkv, block_size, D), gen, torch.bfloat16)
     v = _randn((total, Hkv, block_size, D), gen, torch.bfloat16)
@@ -134,9 +139,10 @@ def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_
         last = int(table[b, nblk[b] - 1])
         k[last, :, tail:] = float("nan")
         v[last, :, tail:] = float("nan")
-    for blk in perm[used:]:
-        k[int(blk)] = float("nan")
-        v[int(blk)] = float("nan")
+    if used < total:
+        idx = torch.from_numpy(perm[used:].astype(np.int64)).to(k.device)
+        k[idx] = float("nan")
+        v[idx] = float("nan")
     return {"q": q, "k_cache": k, "v_cache": v, "seqlens": torch.from_numpy(lens),
             "block_table": torch.from_numpy(table), "block_size": block_size,
             "max_seqlen": int(lens.max(initial=0)), "num_blocks": total}

@@ -95,16 +95,17 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
  *   o           [B, Hq, D] bf16, written
  *   lse         [B, Hq] float32, written; may be NULL
  *
- * max_seqlen must be >= every seqlens[b]; it sizes the split plan and the
- * workspace.  The work is split along the KV length into chunks (attn_decode_plan);
- * each split writes a partial (O, LSE) into `workspace` and a combine pass merges
- * them with the same LSE-weighted rule as the pages' two-way online-softmax merge.
- * The last split of a (sequence, head group) to finish performs that merge, so one
- * kernel launch does the whole decode; a sequence that fits one split is written
- * directly.  workspace must be device memory of at least
+ * max_seqlen must be >= every seqlens[b]; it bounds the workspace.  The work is
+ * split along the KV length (attn_decode_plan, attn_decode_schedule): a persistent grid
+ * of CTAs cuts the token streams of all (sequence, KV head) pairs, laid end to end, into
+ * equal ranges, so every CTA reads the same number of bytes.  A stream shared by several
+ * CTAs yields one partial (O, LSE) per CTA in `workspace`; the CTA that finishes the
+ * stream last merges them with the same LSE-weighted rule as the pages' two-way
+ * online-softmax merge, so one kernel launch does the whole decode.  A stream that lies
+ * within one CTA is written directly.  workspace must be device memory of at least
  * attn_decode_workspace_bytes(...) bytes, 256-byte aligned, and zero-filled before its
  * first use: it holds a sticky error word (read and cleared by attn_decode_check),
- * per-group split counters that each call returns to zero, and the partials.  After a
+ * per-stream merge counters that each call returns to zero, and the partials.  After a
  * call that raised ATTN_DEV_WAIT_TIMEOUT, zero it again.  Calls that share a workspace
  * must not run concurrently.  Device-side
  * checks: a block id outside [0, num_blocks), a seqlen above max_seqlen or above
@@ -155,15 +156,28 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
 size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen);
 
 /* Split-KV plan (pure host function, no device access):
- *   G          = largest of 8, 4, 2, 1 dividing g = Hq/Hkv (query heads per CTA);
- *   streams    = B * Hkv * (g / G);
- *   splits     = clamp(ceil(1184 / streams), 1, min(128, max(1, ceil(max_seqlen / 512))));
- *   chunk      = max(64, 64 * ceil(ceil(max(max_seqlen,1) / splits) / 64)) tokens;
- *   max_splits = max(1, ceil(max_seqlen / chunk)).
- * Sequence b uses ceil(seqlens[b] / chunk) splits (0 when empty).  Any output pointer
- * may be NULL.  Returns ATTN_OK, ATTN_ERR_ARG or ATTN_ERR_HEADS. */
-int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen,
-                     int* chunk_tokens, int* max_splits, int* heads_per_cta);
+ *   G       = largest of 8, 4, 2, 1 dividing g = Hq/Hkv (query heads per CTA);
+ *   Y       = Hkv * (g / G) streams per sequence;
+ *   U_max   = B * Y * ceil(max_seqlen / 16) units of 16 tokens at most;
+ *   ctas    = min(2 * num_sms, 512, max(1, ceil(U_max / 8))).
+ * attn_decode launches `ctas` CTAs, num_sms being the current device's SM count.  Any
+ * output pointer may be NULL.  Returns ATTN_OK, ATTN_ERR_ARG (also when U_max >= 2^52) or
+ * ATTN_ERR_HEADS. */
+int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int num_sms,
+                     int* ctas, int* heads_per_cta);
+
+/* The segments CTA `cta` of a decode launch with `ctas` CTAs processes (pure host
+ * function; seqlens_host are host ints, clamped to [0, max_seqlen] as the kernel does).
+ * With U = Y * sum_b ceil(seqlens[b] / 16) units laid out sequence-major, then stream,
+ * then unit, n = min(ctas, ceil(U / 8)) CTAs receive work and CTA i < n owns units
+ * [floor(i U / n), floor((i+1) U / n)).  Each segment is written as 6 ints:
+ *   b, y (stream: kv_head * (g / G) + subgroup), first token, end token,
+ *   slot (-1: the stream lies wholly in this CTA; 0 or 1: the CTA's partial slot),
+ *   nsplit (number of CTAs sharing the stream).
+ * At most max_segs segments are written to segs; *nseg receives the total count.
+ * Returns ATTN_OK, ATTN_ERR_ARG or ATTN_ERR_HEADS. */
+int attn_decode_schedule(const int* seqlens_host, int B, int Hq, int Hkv, int max_seqlen,
+                         int ctas, int cta, int* segs, int max_segs, int* nseg);
 
 /* Synchronises `stream`, reads the sticky error word in `workspace`, clears it, and
  * returns ATTN_ERR_DEVICE if a decode call since the last check flagged an error
@@ -186,8 +200,8 @@ int attn_device_status(int clear, void* stream);
  * never traps.  Returns the launch status. */
 int attn_selftest_wait_timeout(unsigned long long timeout_ns, void* stream);
 
-/* Test hook for the FMA-pipe exp2 the prefill kernel uses for part of its
- * exponentials: y[i] = 2^x[i] by range reduction to [-1/2, 1/2] and a degree-3
+/* Test hook for an FMA-pipe exp2 (an alternative to the MUFU ex2 for kernels that
+ * are bound by the exponential unit): y[i] = 2^x[i] by range reduction to [-1/2, 1/2] and a degree-3
  * minimax polynomial (max relative error 7.5e-5 for x >= -126; below that the result
  * is a tiny positive number).  x and y are n floats of device memory.  Returns the
  * launch status. */

@@ -36,7 +36,7 @@ from .attention import (
     allowed_mask,
 )
 from .kvcache import kv_cache_bytes_ref, paged_pool_blocks_ref
-from .plan import decode_plan_ref, decode_heads_per_cta_ref
+from .plan import decode_plan_ref, decode_heads_per_cta_ref, decode_schedule_ref
 
 __all__ = [
     "attention_ref",
@@ -48,5 +48,6 @@ __all__ = [
     "kv_cache_bytes_ref",
     "paged_pool_blocks_ref",
     "decode_plan_ref",
+    "decode_schedule_ref",
     "decode_heads_per_cta_ref",
 ]

@@ -1,27 +1,43 @@
-"""Restatement of the library's split-KV decode plan, for bit-exact bookkeeping checks.
+"""Restatement of the library's split-KV decode plan and schedule, for bit-exact checks.
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
-The plan is a scheduling choice of this library (the pages give none); it is
-restated here from the formula documented beside ``attn_decode_plan`` in the C
-header so that tests can compare the two integer for integer.  Any plan gives the
-same attention result; the decode parity tests check that.
+The plan and schedule are scheduling choices of this library (the pages give none);
+they are restated here from the formulas documented beside ``attn_decode_plan`` and
+``attn_decode_schedule`` in the C header so that tests can compare the two integer for
+integer.  Any schedule gives the same attention result; the decode parity tests check
+that.  The restatement below works by interval intersection over the whole unit line,
+not by the library's per-CTA walk, so the two are independent formulations.
+
+Plan:
 
 * heads per CTA ``G``: the largest of 8, 4, 2, 1 that divides ``g = Hq / Hkv``;
-* independent streams ``U = B * Hkv * (g / G)``;
-* splits wanted ``ceil(TARGET_CTAS / U)`` with ``TARGET_CTAS = 1184``, clamped to
-  ``[1, min(128, max(1, ceil(max_seqlen / 512)))]``;
-* ``chunk = 64 * ceil(ceil(max_seqlen / splits) / 64)`` tokens per split (at least 64);
-* ``max_splits = max(1, ceil(max_seqlen / chunk))``;
-* sequence ``b`` uses ``ceil(seqlen_b / chunk)`` splits.
+* streams per sequence ``Y = Hkv * (g / G)``;
+* ``U_max = B * Y * ceil(max_seqlen / 16)``;
+* ``ctas = min(2 * num_sms, 512, max(1, ceil(U_max / 8)))``.
+
+Schedule, for host lengths clamped to ``[0, max_seqlen]``:
+
+* stream ``(b, y)`` holds ``ceil(len_b / 16)`` units; streams are laid out in order of
+  ``b``, then ``y``; ``U`` is the total;
+* ``n = min(ctas, ceil(U / 8))`` CTAs get work; CTA ``i`` owns units
+  ``[floor(i U / n), floor((i + 1) U / n))``;
+* each stream that meets a CTA's range gives that CTA one segment: the tokens of the
+  intersection, ``slot`` -1 when the range holds the whole stream, else 0 when the stream
+  is the CTA's first and 1 otherwise, and ``nsplit`` = the number of CTAs whose ranges
+  meet the stream.
 """
 
 from __future__ import annotations
 
-__all__ = ["decode_plan_ref", "decode_heads_per_cta_ref", "TARGET_CTAS"]
+import bisect
 
-TARGET_CTAS = 1184
-MAX_SPLITS = 128
+__all__ = ["decode_plan_ref", "decode_heads_per_cta_ref", "decode_schedule_ref", "UNIT_TOKENS", "MAX_CTAS"]
+
+UNIT_TOKENS = 16
+MIN_UNITS_PER_CTA = 8
+CTAS_PER_SM = 2
+MAX_CTAS = 512
 
 
 def _cdiv(a: int, b: int) -> int:
@@ -36,15 +52,50 @@ def decode_heads_per_cta_ref(hq: int, hkv: int) -> int:
     return 1
 
 
-def decode_plan_ref(batch: int, hq: int, hkv: int, max_seqlen: int):
-    """Return ``(chunk_tokens, max_splits, heads_per_cta)``."""
+def _streams_per_seq(hq: int, hkv: int) -> int:
+    return hkv * ((hq // hkv) // decode_heads_per_cta_ref(hq, hkv))
+
+
+def decode_plan_ref(batch: int, hq: int, hkv: int, max_seqlen: int, num_sms: int):
+    """Return ``(ctas, heads_per_cta)``."""
     if batch <= 0 or hkv <= 0 or hq <= 0 or hq % hkv or max_seqlen < 0:
         raise ValueError("bad decode plan arguments")
-    g = hq // hkv
-    G = decode_heads_per_cta_ref(hq, hkv)
-    streams = batch * hkv * (g // G)
-    splits = _cdiv(TARGET_CTAS, streams)
-    splits = max(1, min(splits, max(1, _cdiv(max_seqlen, 512)), MAX_SPLITS))
-    chunk = max(64, 64 * _cdiv(_cdiv(max(max_seqlen, 1), splits), 64))
-    max_splits = max(1, _cdiv(max_seqlen, chunk))
-    return chunk, max_splits, G
+    umax = batch * _streams_per_seq(hq, hkv) * _cdiv(max_seqlen, UNIT_TOKENS)
+    cap = min(MAX_CTAS, max(1, _cdiv(umax, MIN_UNITS_PER_CTA)))
+    return max(1, min(cap, CTAS_PER_SM * max(1, num_sms))), decode_heads_per_cta_ref(hq, hkv)
+
+
+def decode_schedule_ref(seqlens, hq: int, hkv: int, max_seqlen: int, ctas: int):
+    """Segments of every CTA: a list (one entry per launched CTA) of lists of
+    ``(b, y, tok0, tok1, slot, nsplit)``."""
+    lens = [min(max(int(x), 0), max_seqlen) for x in seqlens]
+    Y = _streams_per_seq(hq, hkv)
+    streams = []  # (b, y, first unit, end unit, length)
+    pos = 0
+    for b, length in enumerate(lens):
+        units = _cdiv(length, UNIT_TOKENS)
+        for y in range(Y):
+            streams.append((b, y, pos, pos + units, length))
+            pos += units
+    total = pos
+    n = min(ctas, _cdiv(total, MIN_UNITS_PER_CTA))
+    starts = [i * total // n for i in range(n)]
+    ends = [(i + 1) * total // n for i in range(n)]
+    out = [[] for _ in range(ctas)]
+    for b, y, s0, s1, length in streams:
+        if s0 == s1:
+            continue
+        # CTAs whose ranges meet [s0, s1): from the last range starting at or before s0
+        # to the last range starting before s1.
+        i0 = bisect.bisect_right(starts, s0) - 1
+        i1 = bisect.bisect_left(starts, s1) - 1
+        for i in range(i0, i1 + 1):
+            lo, hi = starts[i], ends[i]
+            a, e = max(lo, s0), min(hi, s1)
+            assert a < e
+            whole = lo <= s0 and s1 <= hi
+            slot = -1 if whole else (0 if not out[i] else 1)
+            tok0 = (a - s0) * UNIT_TOKENS
+            tok1 = min(length, (e - s0) * UNIT_TOKENS)
+            out[i].append((b, y, tok0, tok1, slot, 1 if whole else i1 - i0 + 1))
+    return out

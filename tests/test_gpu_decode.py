@@ -1,7 +1,8 @@
 """Decode parity: split-KV decode through the C ABI against the fp64 oracle.
 
 Covers contiguous and paged caches, ragged lengths (1 token, page tails, lengths not
-a multiple of the split chunk), odd page sizes, unused NaN-filled pool blocks, MHA /
+a multiple of the 16-token split unit), the extremes of the balanced schedule (one
+sequence over every CTA, many whole sequences per CTA), odd page sizes, unused NaN-filled pool blocks, MHA /
 GQA / MQA head sharing, D=64 and 128, empty sequences, the device-side block-id check,
 and the two full-size workloads on every output.
 """
@@ -65,6 +66,22 @@ def test_paged_small(cuda_lib, shape):
     x = decode_paged_inputs(B, Hq, Hkv, D, bs, 0, max(lens), seed=bs + B, seqlens=lens, extra_blocks=extra)
     o, lse = _run(x)
     compare(o, lse, *_ref(x), BF16_TOL, f"paged {shape}")
+
+
+@pytest.mark.parametrize("case", [
+    # B, Hq, Hkv, D, lengths: extremes of the balanced schedule
+    (1, 32, 8, 128, [100000]),                       # one sequence spread over every CTA
+    (5, 64, 8, 64, [0, 20000, 0, 1, 7000]),          # empty streams between long ones, G = 8
+    (200, 8, 2, 64, "short"),                        # many whole streams per CTA
+    (3, 32, 32, 128, [4096, 1, 2049]),               # MHA: 96 streams
+])
+def test_schedule_extremes(cuda_lib, case):
+    B, Hq, Hkv, D, lens = case
+    if lens == "short":
+        lens = np.random.Generator(np.random.PCG64(9)).integers(0, 41, size=B).tolist()
+    x = decode_contiguous_inputs(B, Hq, Hkv, D, max(max(lens), 1), 0, 0, seed=B + Hq, seqlens=lens)
+    o, lse = _run(x)
+    compare(o, lse, *_ref(x), BF16_TOL, f"schedule {case[:4]}")
 
 
 def test_empty_sequence_gives_zero_and_neg_inf(cuda_lib):

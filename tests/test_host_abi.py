@@ -30,7 +30,7 @@ def test_exports_every_declared_function(lib):
     assert len(names) >= 10
     for n in names:
         assert hasattr(lib, n), f"{n} declared in include/attn.h but not exported"
-    assert lib.attn_abi_version() == 1
+    assert lib.attn_abi_version() == 2
 
 
 def test_error_strings(lib):
@@ -72,16 +72,39 @@ def test_decode_plan_bit_exact_vs_restatement(lib):
         g = int(rng.choice([1, 2, 3, 4, 5, 6, 8, 16, 32]))
         cases.append((int(rng.integers(1, 300)), hkv * g, hkv, int(rng.integers(0, 200000))))
     for B, hq, hkv, L in cases:
-        assert _lib.decode_plan(B, hq, hkv, L) == oracle.decode_plan_ref(B, hq, hkv, L), (B, hq, hkv, L)
+        for sms in (1, 148, 132, 400):
+            assert _lib.decode_plan(B, hq, hkv, L, sms) == oracle.decode_plan_ref(B, hq, hkv, L, sms), \
+                (B, hq, hkv, L, sms)
+
+
+def test_decode_schedule_bit_exact_vs_restatement(lib):
+    rng = np.random.Generator(np.random.PCG64(3))
+    cases = [(rng.integers(1024, 4097, size=16).tolist(), 32, 8, 4096, 296),
+             (rng.integers(512, 8193, size=64).tolist(), 32, 8, 8192, 296),
+             (rng.integers(512, 8193, size=64).tolist(), 32, 32, 8192, 296),
+             (rng.integers(512, 8193, size=64).tolist(), 32, 1, 8192, 296),
+             ([100000], 64, 8, 100000, 512), ([0, 3, 0, 0, 40], 4, 2, 40, 7), ([0], 4, 4, 0, 296),
+             ([9000, -5, 12], 8, 2, 100, 5)]  # clamped lengths
+    for _ in range(30):
+        B = int(rng.integers(1, 50))
+        L = int(rng.integers(0, 30000))
+        hkv = int(rng.choice([1, 2, 8]))
+        cases.append((rng.integers(0, L + 1, size=B).tolist(), hkv * int(rng.choice([1, 3, 4, 16])), hkv, L,
+                      int(rng.integers(1, 513))))
+    for lens, hq, hkv, L, ctas in cases:
+        ref = oracle.decode_schedule_ref(lens, hq, hkv, L, ctas)
+        for cta in range(ctas):
+            assert _lib.decode_schedule(lens, hq, hkv, L, ctas, cta) == ref[cta], (lens[:4], hq, hkv, L, ctas, cta)
 
 
 def test_decode_workspace_bytes_formula(lib):
-    for B, hq, hkv, d, L in [(16, 32, 8, 128, 4096), (64, 32, 8, 128, 8192), (1, 4, 1, 64, 10)]:
-        chunk, ms, G = oracle.decode_plan_ref(B, hq, hkv, L)
+    for B, hq, hkv, d, L in [(16, 32, 8, 128, 4096), (64, 32, 8, 128, 8192), (1, 4, 1, 64, 10),
+                             (1, 32, 32, 64, 0)]:
+        cap, G = oracle.decode_plan_ref(B, hq, hkv, L, 10 ** 6)  # the bound that does not depend on the device
+        Y = hkv * (hq // hkv // G)
         r256 = lambda n: -(-n // 256) * 256
-        cnt_bytes = r256(B * hkv * (hq // hkv // G) * 4)
-        lse_bytes = r256(B * hq * ms * 4)
-        assert _lib.decode_workspace_bytes(B, hq, hkv, d, L) == 256 + cnt_bytes + lse_bytes + B * hq * ms * d * 4
+        assert _lib.decode_workspace_bytes(B, hq, hkv, d, L) == (256 + r256(B * Y * 4) + r256(cap * 2 * G * 4)
+                                                                 + cap * 2 * G * d * 4)
     assert _lib.decode_workspace_bytes(0, 1, 1, 64, 1) == 0
 
 

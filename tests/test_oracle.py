@@ -31,6 +31,8 @@ from oracle import (
     kv_cache_bytes_ref,
     paged_pool_blocks_ref,
     decode_plan_ref,
+    decode_heads_per_cta_ref,
+    decode_schedule_ref,
 )
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -392,9 +394,69 @@ def test_planted_top_left_causal_is_caught(monkeypatch):
                                   (2, 6, 2, 0), (128, 64, 8, 300)])
 def test_decode_plan_invariants(args):
     B, Hq, Hkv, L = args
-    chunk, ms, G = decode_plan_ref(B, Hq, Hkv, L)
-    assert chunk % 64 == 0 and chunk >= 64
-    assert ms >= 1 and chunk * ms >= L
-    assert (Hq // Hkv) % G == 0 and G in (1, 2, 4, 8)
-    if L > 0:
-        assert chunk * (ms - 1) < L  # no split is empty at the maximum length
+    for sms in (1, 148, 1000):
+        ctas, G = decode_plan_ref(B, Hq, Hkv, L, sms)
+        assert (Hq // Hkv) % G == 0 and G in (1, 2, 4, 8)
+        assert 1 <= ctas <= min(2 * sms, 512)
+        units = B * Hkv * (Hq // Hkv // G) * -(-L // 16)
+        assert ctas <= max(1, -(-units // 8))
+
+
+def _schedule_cases():
+    rng = np.random.Generator(np.random.PCG64(5))
+    cases = [([2575, 1030, 4096, 1024], 32, 8, 4096, 296),   # config-3-like lengths
+             ([0, 0, 5, 0], 4, 1, 5, 296),                   # mostly empty
+             ([100000], 32, 8, 100000, 296),                 # one long sequence over every CTA
+             ([1, 17, 16, 33], 8, 8, 33, 3),                 # ragged, few CTAs
+             ([0, 0], 4, 2, 10, 8)]                          # nothing to do
+    for _ in range(40):
+        B = int(rng.integers(1, 40))
+        L = int(rng.integers(0, 20000))
+        hkv = int(rng.choice([1, 2, 8]))
+        hq = hkv * int(rng.choice([1, 4, 8, 32]))
+        lens = rng.integers(0, L + 1, size=B).tolist()
+        cases.append((lens, hq, hkv, L, int(rng.integers(1, 600))))
+    return cases
+
+
+@pytest.mark.parametrize("case", _schedule_cases())
+def test_decode_schedule_tiles_every_stream_once(case):
+    """Brute-force check of the schedule restatement: the segments of all CTAs cover every
+    token of every stream exactly once, ranges are balanced to one unit, slots and split
+    counts are consistent."""
+    lens, hq, hkv, L, ctas = case
+    sched = decode_schedule_ref(lens, hq, hkv, L, ctas)
+    assert len(sched) == ctas
+    G = decode_heads_per_cta_ref(hq, hkv)
+    Y = hkv * (hq // hkv // G)
+    cover = {}
+    units_per_cta = []
+    for segs in sched:
+        units = 0
+        for k, (b, y, t0, t1, slot, nsplit) in enumerate(segs):
+            assert 0 <= t0 < t1 <= min(lens[b], L) and t0 % 16 == 0
+            assert (t1 == min(lens[b], L)) or t1 % 16 == 0
+            if slot == 1:
+                assert k == len(segs) - 1 and k > 0  # only the last segment can be a second partial
+            if slot == 0:
+                assert k == 0
+            if 0 < k < len(segs) - 1:
+                assert slot == -1  # middle segments are whole streams
+            units += -(-(t1 - t0) // 16)
+            cover.setdefault((b, y), []).append((t0, t1, slot, nsplit))
+        units_per_cta.append(units)
+    for b, n in enumerate(lens):
+        for y in range(Y):
+            n = min(max(n, 0), L)
+            pieces = sorted(cover.get((b, y), []))
+            if n == 0:
+                assert not pieces
+                continue
+            assert pieces[0][0] == 0 and pieces[-1][1] == n
+            assert all(pieces[i][1] == pieces[i + 1][0] for i in range(len(pieces) - 1))
+            assert all(p[3] == len(pieces) for p in pieces)
+            assert (len(pieces) == 1) == (pieces[0][2] == -1)
+    busy = [u for u in units_per_cta if u > 0]
+    if busy:
+        # a segment's unit count is exact (t0 is unit-aligned, t1 aligned or the sequence end)
+        assert max(busy) - min(busy) <= 1

@@ -42,12 +42,16 @@ def test_noalloc_matches_workspace_decode_on_two_calls(cuda_lib, kind):
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch(cuda_lib):
-    # 1024 sequences x 32 heads x 128 dims of fp32 partials alone exceed 16 MiB.
-    B, Hq, Hkv, D, L = 1024, 32, 8, 128, 8192
+    # 65535 sequences x 64 KV heads need 16.8 MB of merge counters alone, above 16 MiB.
+    # The request is refused from its sizes before any pointer is used, so small buffers
+    # viewed with the large shapes stand in for the inputs.
+    B, Hq, Hkv, D, L = 65535, 64, 64, 128, 16
     assert _lib.decode_workspace_bytes(B, Hq, Hkv, D, L) > _lib.DECODE_NOALLOC_SCRATCH_BYTES
-    q = torch.zeros(B, Hq, D, dtype=torch.bfloat16, device="cuda")
-    kc = torch.zeros(B, Hkv, 16, D, dtype=torch.bfloat16, device="cuda")
-    seqlens = torch.ones(B, dtype=torch.int32, device="cuda")
+    q = torch.zeros(1, 1, D, dtype=torch.bfloat16, device="cuda").expand(B, Hq, D)
+    kc = torch.zeros(1, 1, 16, D, dtype=torch.bfloat16, device="cuda").expand(B, Hkv, 16, D)
+    seqlens = torch.ones(1, dtype=torch.int32, device="cuda").expand(B)
+    o = torch.zeros(1, 1, D, dtype=torch.bfloat16, device="cuda").expand(B, Hq, D)
+    lse = torch.zeros(1, 1, dtype=torch.float32, device="cuda").expand(B, Hq)
     with pytest.raises(_lib.AttnError) as e:
-        _lib.attn_decode_noalloc(q, kc, kc, seqlens, max_seqlen=L)
+        _lib.attn_decode_noalloc(q, kc, kc, seqlens, max_seqlen=L, o=o, lse=lse)
     assert e.value.status == _lib.ATTN_ERR_SCRATCH_LIMIT
