@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -83,6 +84,19 @@ __global__ void fill_empty_rows_kernel(float* lse, size_t n) {
   if (i < n) lse[i] = -INFINITY;
 }
 
+// SM count of the current device, looked up once per device.
+int device_sms() {
+  static int sms[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    sms[dev] = v;
+  }
+  return sms[dev];
+}
+
 template <int D>
 int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Sq, int Sk, float scale, int causal, cudaStream_t st) {
@@ -109,7 +123,10 @@ int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* l
   const long long items_b = (long long)p.npq * B * Hkv;
   if (items_a + items_b > INT_MAX) return ATTN_ERR_UNSUPPORTED;
   p.items_a = (int)items_a;
-  const int grid = (int)(items_a + items_b);
+  p.items = (int)(items_a + items_b);
+  const int sms = device_sms();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const int grid = std::min(p.items, sms);  // persistent: one CTA per SM walks its share of the items
   auto kern = attn::tc::fwd_tc_kernel<D>;
   cudaError_t e = set_smem_once(kern, Lay::kAlloc, D == 64 ? 0 : 1);
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
@@ -153,19 +170,6 @@ bool decode_plan(int B, int Hq, int Hkv, int max_seqlen, DecodePlan* out) {
 
 inline int plan_ctas(const DecodePlan& pl, int num_sms) {
   return std::max(1, std::min(pl.ctas_cap, attn::dec::kCtasPerSm * std::max(1, num_sms)));
-}
-
-// SM count of the current device, looked up once per device.
-int device_sms() {
-  static int sms[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (sms[dev] == 0) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-    sms[dev] = v;
-  }
-  return sms[dev];
 }
 
 inline size_t round256(size_t n) { return (n + 255) & ~size_t(255); }

@@ -10,8 +10,11 @@
 //    query heads of one KV group at the same positions (GQA: one K/V tile load serves
 //    both heads), or, when the group has an odd head left over, two consecutive query
 //    tiles of that head.
-//  * warp 0 (one thread) streams Q once and K/V tiles of 128 keys through a 2-stage
-//    shared-memory ring with TMA (128-byte swizzle).
+//  * warp 0 (one thread) streams Q once and the K and V tiles of 128 keys, in the order
+//    K_0, V_0, K_1, V_1, ..., through one 5-slot shared-memory ring with TMA (128-byte
+//    swizzle).  Each slot is released as soon as the MMAs that read it complete, so a
+//    tile is requested about two KV steps before it is needed: under load an L2-resident
+//    tile takes of the order of two microseconds to arrive.
 //  * warp 1 (one thread) issues the tcgen05 MMAs: S_i = Q_i K^T (A, B from shared
 //    memory) into TMEM, and O_i += P_i V with P_i read from TMEM (it overwrites S_i as
 //    bf16).  The issue order PV_0, S_0, PV_1, S_1 makes each slot's softmax overlap the
@@ -42,14 +45,15 @@ namespace tc {
 constexpr int BM = 128;  // query rows per tile (MMA M)
 constexpr int BN = 128;  // keys per K/V tile
 constexpr int kThreads = 384;
+constexpr int kRingStages = 5;  // K/V ring slots (with the two Q tiles: 7 x 32 KB at D=128)
 // Register split (setmaxnreg): the launch gives every thread 168 registers (65536 / 384
 // rounded down to a multiple of 8), i.e. 64512 in total.  Warpgroup 0 (TMA, MMA, two
 // idle warps) gives registers to the two softmax warpgroups; the split per
-// head dim is the one with the fewest spills (D=128: 64 * 128 + 216 * 256 = 63488;
+// head dim is the one with the fewest spills (D=128: 72 * 128 + 216 * 256 = 64512;
 // D=64: 56 * 128 + 224 * 256 = 64512).
 template <int D>
 struct Regs {
-  static constexpr int kControl = D == 128 ? 64 : 56;
+  static constexpr int kControl = D == 128 ? 72 : 56;
   static constexpr int kSoftmax = D == 128 ? 216 : 224;
 };
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
@@ -60,29 +64,29 @@ struct Layout {
   static constexpr int kTile = BM * D * 2;  // bytes of one Q, K or V tile (BN == BM)
   static constexpr int kBox = BM * 128;     // bytes of one 64-column TMA box
   static constexpr int kQ = 0;              // Q[2]
-  static constexpr int kK = 2 * kTile;      // K[2]
-  static constexpr int kV = 4 * kTile;      // V[2]
-  static constexpr int kBar = 6 * kTile;
-  static constexpr int kNumBars = 20;
+  static constexpr int kRing = 2 * kTile;   // K/V ring[kRingStages]
+  static constexpr int kBar = (2 + kRingStages) * kTile;
+  static constexpr int kNumBars = 2 + 2 * kRingStages + 12;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
+  static_assert(kAlloc <= 232448, "dynamic shared memory per CTA on sm_100 is at most 227 KB");
   static constexpr uint32_t kColS0 = 0, kColS1 = BN, kColO0 = 2 * BN, kColO1 = 2 * BN + D;
   static constexpr uint32_t kTmemCols = 512;
 };
 
 // barrier indices
 enum : int {
-  kBarQ = 0,
-  kBarKFull = 1,   // [2] TMA bytes landed
-  kBarKEmpty = 3,  // [2] MMAs that read the stage have completed
-  kBarVFull = 5,   // [2]
-  kBarVEmpty = 7,  // [2]
-  kBarSFull = 9,   // [2] per slot: S_i written
-  kBarP0 = 11,     // [2] per slot: P_i keys 0..63 written, O_i rescaled (128 arrivals)
-  kBarP1 = 13,     // [2] per slot: P_i keys 64..127 written (128 arrivals)
-  kBarODone = 15,  // [2] per slot: PV_i finished
-  kBarDrain = 17,  // used only when giving up
+  kBarQFull = 0,                          // the item's Q tiles landed
+  kBarQEmpty = 1,                         // the item's S MMAs are done with the Q tiles
+  kBarFull = 2,                           // [kRingStages] TMA bytes of a ring slot landed
+  kBarEmpty = kBarFull + kRingStages,     // [kRingStages] MMAs that read the slot have completed
+  kBarSFull = kBarEmpty + kRingStages,    // [2] per slot: S_i written
+  kBarP0 = kBarSFull + 2,                 // [2] per slot: P_i keys 0..63 written, O_i rescaled (128 arrivals)
+  kBarP1 = kBarP0 + 2,                    // [2] per slot: P_i keys 64..127 written (128 arrivals)
+  kBarODone = kBarP1 + 2,                 // [2] per slot: PV_i finished
+  kBarOFree = kBarODone + 2,              // [2] per slot: O_i read out by the epilogue (128 arrivals)
+  kBarDrain = kBarOFree + 2,              // used only when giving up
 };
 
 struct Params {
@@ -95,6 +99,7 @@ struct Params {
   int pairs;        // head pairs per KV group (g / 2)
   int items_a;      // work items made of head pairs
   int npq;          // query-tile pairs of the leftover head when g is odd
+  int items;        // all work items
 };
 
 struct Item {
@@ -195,20 +200,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const Item it = decode_item(p, blockIdx.x);
-  const int N = max(it.n[0], it.n[1]);
+  // Persistent CTAs: round r of the longest-first item list gives CTA c item r*C + c on even
+  // rounds and r*C + (C-1-c) on odd ones (a snake, so the long and short items even out).
+  // Every role walks the same list; items without work for the MMAs are skipped by the
+  // producer and the issuer alike.
+  const int C = (int)gridDim.x;
+  auto item_of = [&](int r) -> int { return r * C + ((r & 1) ? C - 1 - (int)blockIdx.x : (int)blockIdx.x); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kBarQ), 1);
+    mbar_init(bar(kBarQFull), 1);
+    mbar_init(bar(kBarQEmpty), 1);
+    for (int s = 0; s < kRingStages; ++s) {
+      mbar_init(bar(kBarFull + s), 1);
+      mbar_init(bar(kBarEmpty + s), 1);
+    }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
-      mbar_init(bar(kBarVFull + s), 1);
-      mbar_init(bar(kBarVEmpty + s), 1);
       mbar_init(bar(kBarSFull + s), 1);
       mbar_init(bar(kBarP0 + s), 128);
       mbar_init(bar(kBarP1 + s), 128);
       mbar_init(bar(kBarODone + s), 1);
+      mbar_init(bar(kBarOFree + s), 128);
       mbar_init(bar(kBarDrain + s), 1);
     }
     *abort_flag = 0;
@@ -228,46 +239,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const uint32_t sQ0 = sbase + L::kQ, sK0 = sbase + L::kK, sV0 = sbase + L::kV;
+  const uint32_t sQ0 = sbase + L::kQ, sR0 = sbase + L::kRing;
+  // Ring positions run on across items: an item whose first position is b puts K_j at b + 2j and
+  // V_j at b + 2j + 1; slot = position % kRingStages, fill = position / kRingStages.
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(Regs<D>::kControl));
     if (warp == 0) {
       // ---------------------------------------------------------- TMA producer
-      if (lane == 0 && N > 0) {
-        int k_fill[2] = {-1, -1}, v_fill[2] = {-1, -1};
-        uint32_t qbytes = 0;
-        for (int i = 0; i < 2; ++i) qbytes += it.n[i] > 0 ? (uint32_t)L::kTile : 0u;
-        mbar_arrive_expect_tx(bar(kBarQ), qbytes);
-        for (int i = 0; i < 2; ++i) {
-          if (it.n[i] == 0) continue;
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ0 + i * L::kTile + c * L::kBox, &tmQ, bar(kBarQ), c * 64, it.t[i] * BM,
-                        it.b * p.Hq + it.h[i]);
-        }
-        const int zkv = it.b * p.Hkv + it.kvh;
-        for (int j = 0; j < N; ++j) {
-          const int s = j & 1;
-          const int f = j >> 1;
-          if (f > 0 && !mbar_wait(bar(kBarKEmpty + s), (f - 1) & 1, abort_flag)) break;
-          mbar_arrive_expect_tx(bar(kBarKFull + s), L::kTile);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sK0 + s * L::kTile + c * L::kBox, &tmK, bar(kBarKFull + s), c * 64, j * BN, zkv);
-          k_fill[s] = f;
-          if (f > 0 && !mbar_wait(bar(kBarVEmpty + s), (f - 1) & 1, abort_flag)) break;
-          mbar_arrive_expect_tx(bar(kBarVFull + s), L::kTile);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sV0 + s * L::kTile + c * L::kBox, &tmV, bar(kBarVFull + s), c * 64, j * BN, zkv);
-          v_fill[s] = f;
+      if (lane == 0) {
+        int fill[kRingStages];
+        for (int s = 0; s < kRingStages; ++s) fill[s] = -1;
+        int qn = 0, pos = 0;
+        bool alive = true;
+        for (int r = 0; alive; ++r) {
+          const int idx = item_of(r);
+          if (idx >= p.items) break;
+          const Item it = decode_item(p, idx);
+          const int N = max(it.n[0], it.n[1]);
+          if (N == 0) continue;
+          // Q of this item replaces the previous item's once its S MMAs are done.
+          if (qn > 0 && !mbar_wait(bar(kBarQEmpty), (qn - 1) & 1, abort_flag)) break;
+          uint32_t qbytes = 0;
+          for (int i = 0; i < 2; ++i) qbytes += it.n[i] > 0 ? (uint32_t)L::kTile : 0u;
+          mbar_arrive_expect_tx(bar(kBarQFull), qbytes);
+          for (int i = 0; i < 2; ++i) {
+            if (it.n[i] == 0) continue;
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sQ0 + i * L::kTile + c * L::kBox, &tmQ, bar(kBarQFull), c * 64, it.t[i] * BM,
+                          it.b * p.Hq + it.h[i]);
+          }
+          ++qn;
+          const int zkv = it.b * p.Hkv + it.kvh;
+          for (int k = 0; k < 2 * N; ++k, ++pos) {
+            const int s = pos % kRingStages;
+            const int f = pos / kRingStages;
+            if (f > 0 && !mbar_wait(bar(kBarEmpty + s), (f - 1) & 1, abort_flag)) {
+              alive = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(kBarFull + s), L::kTile);
+            const void* tm = (k & 1) ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
+            for (int c = 0; c < D / 64; ++c)
+              tma_load_3d(sR0 + s * L::kTile + c * L::kBox, tm, bar(kBarFull + s), c * 64, (k >> 1) * BN, zkv);
+            fill[s] = f;
+          }
         }
         if (*abort_flag) {
           // Let copies already in flight land before the CTA's shared memory is released.
           int never = 0;
-          mbar_wait(bar(kBarQ), 0, &never, 100000000ull);
-          for (int s = 0; s < 2; ++s) {
-            if (k_fill[s] >= 0) mbar_wait(bar(kBarKFull + s), k_fill[s] & 1, &never, 100000000ull);
-            if (v_fill[s] >= 0) mbar_wait(bar(kBarVFull + s), v_fill[s] & 1, &never, 100000000ull);
-          }
+          if (qn > 0) mbar_wait(bar(kBarQFull), (qn - 1) & 1, &never, 100000000ull);
+          for (int s = 0; s < kRingStages; ++s)
+            if (fill[s] >= 0) mbar_wait(bar(kBarFull + s), fill[s] & 1, &never, 100000000ull);
         }
       }
     } else if (warp == 1) {
@@ -276,64 +299,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       // thread execute in issue order, so S_i(j+1) may be issued right behind PV_i(j), which
       // reads P_i from the same TMEM columns.  While softmax 0 works on S_0(j+1) the pipe runs
       // slot 1's PV and S, and the other way round.
-      if (lane == 0 && N > 0) {
+      // The whole warp runs this loop with uniform control flow and one elected lane issues
+      // each MMA: the operands are then warp-uniform, and the shared-memory descriptors are
+      // built once and advanced by constant offsets (the start-address field is the low 14
+      // bits, address / 16, and no offset here carries out of it).  The MMA issue rate, not the
+      // tensor pipe, otherwise limits the KV step.
+      {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BN, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, true);
+        const uint64_t qdesc0 = smem_desc_sw128(sQ0, 16, 1024);
+        const uint64_t kdesc0 = smem_desc_sw128(sR0, 16, 1024);
+        // V tile: 128 key rows of 128 bytes per 64-column box; MN-major B operand.
+        const uint64_t vdesc0 = smem_desc_sw128(sR0, L::kBox, 1024);
+        const bool leader = elect_one();
         auto issue_s = [&](int i, int s) {
           tc_fence_after();
-          const uint32_t sQ = sQ0 + i * L::kTile, sK = sK0 + s * L::kTile;
+          const uint64_t qd = qdesc0 + (uint64_t)((i * L::kTile) >> 4);
+          const uint64_t kd = kdesc0 + (uint64_t)((s * L::kTile) >> 4);
           const uint32_t tS = tmem + (i ? L::kColS1 : L::kColS0);
+          if (leader) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (uint32_t)(kk >> 2) * L::kBox + (uint32_t)(kk & 3) * 32u;
-            mma_ss(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idesc_qk,
-                   kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4);
+              mma_ss(tS, qd + off, kd + off, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(bar(kBarSFull + i));
           }
-          tc_commit(bar(kBarSFull + i));
+          __syncwarp();
         };
-        // V tile: 128 key rows of 128 bytes per 64-column box; MN-major B operand.
         auto issue_pv = [&](int i, int s, int j, int k0) {
           tc_fence_after();
-          const uint32_t sV = sV0 + s * L::kTile;
+          const uint64_t vd = vdesc0 + (uint64_t)((s * L::kTile) >> 4);
           const uint32_t tS = tmem + (i ? L::kColS1 : L::kColS0), tO = tmem + (i ? L::kColO1 : L::kColO0);
+          if (leader) {
 #pragma unroll
-          for (int kk = k0; kk < k0 + 4; ++kk)
-            mma_ts(tO, tS + (uint32_t)kk * 8u, smem_desc_sw128(sV + (uint32_t)kk * 2048u, L::kBox, 1024), idesc_pv,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-        };
-        bool ok = mbar_wait(bar(kBarQ), 0, abort_flag) && mbar_wait(bar(kBarKFull), 0, abort_flag);
-        if (ok) {
-          for (int i = 0; i < 2; ++i)
-            if (it.n[i] > 0) issue_s(i, 0);
-          tc_commit(bar(kBarKEmpty));
-        }
-        for (int j = 0; ok && j < N; ++j) {
-          const int s = j & 1, s1 = (j + 1) & 1;
-          bool next_k = false;
-          if (!(ok = mbar_wait(bar(kBarVFull + s), (j >> 1) & 1, abort_flag))) break;
-          for (int i = 0; i < 2; ++i) {
-            const int ni = i ? it.n[1] : it.n[0];
-            if (j >= ni) continue;
-            if (!(ok = mbar_wait(bar(kBarP0 + i), j & 1, abort_flag))) break;
-            issue_pv(i, s, j, 0);
-            if (!(ok = mbar_wait(bar(kBarP1 + i), j & 1, abort_flag))) break;
-            issue_pv(i, s, j, 4);
-            tc_commit(bar(kBarODone + i));
-            if (j + 1 < ni) {
-              if (!next_k) {
-                if (!(ok = mbar_wait(bar(kBarKFull + s1), ((j + 1) >> 1) & 1, abort_flag))) break;
-                next_k = true;
-              }
-              issue_s(i, s1);
-            }
+            for (int kk = k0; kk < k0 + 4; ++kk)
+              mma_ts(tO, tS + (uint32_t)kk * 8u, vd + (uint64_t)((kk * 2048) >> 4), idesc_pv,
+                     (j > 0 || kk > 0) ? 1u : 0u);
           }
-          if (!ok) break;
-          tc_commit(bar(kBarVEmpty + s));
-          if (j + 1 < N) tc_commit(bar(kBarKEmpty + s1));
+          __syncwarp();
+        };
+        auto commit = [&](int b) {
+          if (leader) tc_commit(bar(b));
+          __syncwarp();
+        };
+        auto slot_of = [](int pos) { return pos % kRingStages; };
+        auto phase_of = [](int pos) { return (uint32_t)((pos / kRingStages) & 1); };
+        int qn = 0, pos = 0;
+        int gs[2] = {0, 0};    // KV steps issued per slot so far (phases of SFull, P0, P1, ODone)
+        int done[2] = {0, 0};  // items per slot whose O has been produced (phases of OFree)
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int idx = item_of(r);
+          if (idx >= p.items) break;
+          const Item it = decode_item(p, idx);
+          const int N = max(it.n[0], it.n[1]);
+          if (N == 0) continue;
+          if (!(ok = warp_wait(bar(kBarQFull), qn & 1, abort_flag))) break;
+          if (!(ok = warp_wait(bar(kBarFull + slot_of(pos)), phase_of(pos), abort_flag))) break;
+          // S_i(0) reuses the TMEM of the previous item's P_i: in issue order behind its PV.
+          for (int i = 0; i < 2; ++i)
+            if (it.n[i] > 0) issue_s(i, slot_of(pos));
+          commit(kBarEmpty + slot_of(pos));
+          if (N == 1) commit(kBarQEmpty);
+          for (int j = 0; ok && j < N; ++j) {
+            const int kv = pos + 2 * j + 1, kn = pos + 2 * j + 2;  // ring positions of V_j and K_{j+1}
+            const int last = j < it.n[1] ? 1 : 0;                 // the last slot that multiplies by V_j
+            bool next_k = false;
+            if (!(ok = warp_wait(bar(kBarFull + slot_of(kv)), phase_of(kv), abort_flag))) break;
+            for (int i = 0; i < 2; ++i) {
+              const int ni = i ? it.n[1] : it.n[0];
+              if (j >= ni) continue;
+              const uint32_t ph = (uint32_t)((gs[i] + j) & 1);
+              if (!(ok = warp_wait(bar(kBarP0 + i), ph, abort_flag))) break;
+              // PV_i(0) overwrites O_i: the previous item's epilogue must have read it.
+              if (j == 0 && done[i] > 0 && !(ok = warp_wait(bar(kBarOFree + i), (done[i] - 1) & 1, abort_flag)))
+                break;
+              issue_pv(i, slot_of(kv), j, 0);
+              if (!(ok = warp_wait(bar(kBarP1 + i), ph, abort_flag))) break;
+              issue_pv(i, slot_of(kv), j, 4);
+              commit(kBarODone + i);
+              if (i == last) commit(kBarEmpty + slot_of(kv));  // V_j's slot, once its PVs are done
+              if (j + 1 < ni) {
+                if (!next_k) {
+                  if (!(ok = warp_wait(bar(kBarFull + slot_of(kn)), phase_of(kn), abort_flag))) break;
+                  next_k = true;
+                }
+                issue_s(i, slot_of(kn));
+              }
+            }
+            if (!ok) break;
+            if (j + 1 < N) commit(kBarEmpty + slot_of(kn));
+            if (j + 2 == N) commit(kBarQEmpty);  // every S MMA of the item has been issued
+          }
+          for (int i = 0; i < 2; ++i) {
+            gs[i] += it.n[i];
+            done[i] += it.n[i] > 0 ? 1 : 0;
+          }
+          pos += 2 * N;
+          ++qn;
         }
         if (!ok) {
           int never = 0;
-          tc_commit(bar(kBarDrain));
+          commit(kBarDrain);
           mbar_wait(bar(kBarDrain), 0, &never, 100000000ull);
         }
       }
@@ -344,15 +412,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = (warp - 4) >> 2;  // slot
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;
-    const int n = i ? it.n[1] : it.n[0];
-    const int t = i ? it.t[1] : it.t[0];
-    const int h = i ? it.h[1] : it.h[0];
-    if (t < p.nq) {
-      const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-      const uint32_t tS = tmem + lane_off + (i ? L::kColS1 : L::kColS0);
-      const uint32_t tO = tmem + lane_off + (i ? L::kColO1 : L::kColO0);
-      const uint32_t bar_s = bar(kBarSFull + i), bar_o = bar(kBarODone + i);
-      const uint32_t bar_p0 = bar(kBarP0 + i), bar_p1 = bar(kBarP1 + i);
+    const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + (i ? L::kColS1 : L::kColS0);
+    const uint32_t tO = tmem + lane_off + (i ? L::kColO1 : L::kColO0);
+    const uint32_t bar_s = bar(kBarSFull + i), bar_o = bar(kBarODone + i);
+    const uint32_t bar_p0 = bar(kBarP0 + i), bar_p1 = bar(kBarP1 + i);
+    int gs = 0;  // KV steps of this slot in earlier items (phases of SFull, P0, P1, ODone)
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int idx = item_of(r);
+      if (idx >= p.items) break;
+      const Item it = decode_item(p, idx);
+      const int n = i ? it.n[1] : it.n[0];
+      const int t = i ? it.t[1] : it.t[0];
+      const int h = i ? it.h[1] : it.h[0];
+      if (t >= p.nq) continue;  // this slot has no query tile in the item
       const int qrow = t * BM + row;
       const long long key_limit = p.causal ? (long long)qrow + p.Sk - p.Sq : (long long)p.Sk - 1;
       const long long tile_limit = p.causal ? (long long)t * BM + p.Sk - p.Sq : (long long)p.Sk - 1;
@@ -361,9 +435,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // l: fp32 row sum (for the LSE); lr: row sum of the bf16 P that the tensor core
       // multiplies, so that O / lr uses exactly normalised weights.
       float m = -INFINITY, l = 0.f, lr = 0.f;
-      bool ok = true;
       for (int j = 0; j < n; ++j) {
-        if (!(ok = warp_wait(bar_s, j & 1, abort_flag))) break;
+        if (!(ok = warp_wait(bar_s, (gs + j) & 1, abort_flag))) break;
         tc_fence_after();
         const int kv0 = j * BN;
         // Mask only tiles that reach past the last key or the causal diagonal.
@@ -442,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           exp_chunk(r1, pa + 16, c2, nmu2, acc0, accr0);
           if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
             // O_i must hold PV_i(j-1) before it is rescaled, and be rescaled before PV_i(j).
-            if (!(ok = warp_wait(bar_o, (j - 1) & 1, abort_flag))) break;
+            if (!(ok = warp_wait(bar_o, (gs + j - 1) & 1, abort_flag))) break;
             tc_fence_after();
             const uint64_t a2 = f2pack(alpha, alpha);
 #pragma unroll
@@ -472,9 +545,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         lr = fmaf(lr, alpha, q_lo + q_hi);
       }
       // ---------------------------------------------------------- epilogue
-      if (ok && n > 0) ok = warp_wait(bar_o, (n - 1) & 1, abort_flag);
-      if (ok) {
+      if (!ok) break;
+      uint32_t oe[D / 32][32];
+      if (n > 0) {
+        if (!(ok = warp_wait(bar_o, (gs + n - 1) & 1, abort_flag))) break;
         tc_fence_after();
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4) tmem_ld32(tO + 32u * c4, oe[c4]);
+        tmem_wait_ld();
+        // O_i is in registers: the next item's PV_i may overwrite it.
+        tc_fence_before();
+        mbar_arrive(bar(kBarOFree + i));
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) oe[c4][e] = 0u;
+      }
+      {
         const int bh = it.b * p.Hq + h;
         const bool in_range = qrow < p.Sq;
         const float inv_l = lr > 0.f ? 1.f / lr : 0.f;
@@ -482,14 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             reinterpret_cast<__nv_bfloat16*>(p.o) + ((size_t)bh * p.Sq + (in_range ? qrow : 0)) * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
-          uint32_t ov[32];
-          if (n > 0) {
-            tmem_ld32(tO + 32u * c4, ov);
-            tmem_wait_ld();
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = 0u;
-          }
+          const uint32_t(&ov)[32] = oe[c4];
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
@@ -503,6 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (p.lse != nullptr && in_range)
           p.lse[(size_t)bh * p.Sq + qrow] = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
       }
+      gs += n;
     }
   }
 
