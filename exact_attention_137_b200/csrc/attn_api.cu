@@ -124,6 +124,14 @@ int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* l
   if (items_a + items_b > INT_MAX) return ATTN_ERR_UNSUPPORTED;
   p.items_a = (int)items_a;
   p.items = (int)(items_a + items_b);
+  p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0 ? 1 : 0;
+  p.g = g;
+  using attn::tc::make_fastdiv;
+  p.div_per_t = make_fastdiv((uint32_t)std::max(1LL, (long long)B * Hkv * p.pairs));
+  p.div_hp = make_fastdiv((uint32_t)std::max(1, Hkv * p.pairs));
+  p.div_pairs = make_fastdiv((uint32_t)std::max(1, p.pairs));
+  p.div_bh = make_fastdiv((uint32_t)((long long)B * Hkv));
+  p.div_hkv = make_fastdiv((uint32_t)Hkv);
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = std::min(p.items, sms);  // persistent: one CTA per SM walks its share of the items

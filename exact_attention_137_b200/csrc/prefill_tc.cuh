@@ -49,12 +49,12 @@ constexpr int kRingStages = 5;  // K/V ring slots (with the two Q tiles: 7 x 32 
 // Register split (setmaxnreg): the launch gives every thread 168 registers (65536 / 384
 // rounded down to a multiple of 8), i.e. 64512 in total.  Warpgroup 0 (TMA, MMA, two
 // idle warps) gives registers to the two softmax warpgroups; the split per
-// head dim is the one with the fewest spills (D=128: 72 * 128 + 216 * 256 = 64512;
+// head dim is the one with the fewest spills (D=128: 88 * 128 + 208 * 256 = 64512;
 // D=64: 56 * 128 + 224 * 256 = 64512).
 template <int D>
 struct Regs {
-  static constexpr int kControl = D == 128 ? 72 : 56;
-  static constexpr int kSoftmax = D == 128 ? 216 : 224;
+  static constexpr int kControl = D == 128 ? 88 : 56;
+  static constexpr int kSoftmax = D == 128 ? 208 : 224;
 };
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kFastBound = 64.0f;        // log2 units: fast-path values stay below 2^64
@@ -89,6 +89,28 @@ enum : int {
   kBarDrain = kBarOFree + 2,              // used only when giving up
 };
 
+// Division by a runtime constant d >= 1 for dividends below 2^31: q = (umulhi(x, m) + x) >> s
+// with s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1 (Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994).  The work-item decode runs on
+// the critical path between two items, where a hardware-less 32-bit division costs dozens of
+// instructions.
+struct FastDiv {
+  uint32_t d, m, s;
+};
+
+inline FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f;
+  f.d = d;
+  f.s = 0;
+  while ((1ull << f.s) < d) ++f.s;
+  f.m = (uint32_t)(((1ull << 32) * ((1ull << f.s) - d)) / d + 1);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fdiv(uint32_t x, const FastDiv& f) {
+  return (__umulhi(x, f.m) + x) >> f.s;
+}
+
 struct Params {
   void* o;
   float* lse;
@@ -100,6 +122,13 @@ struct Params {
   int items_a;      // work items made of head pairs
   int npq;          // query-tile pairs of the leftover head when g is odd
   int items;        // all work items
+  int o_align32;    // O's base is 32-byte aligned (256-bit stores allowed)
+  int g;            // Hq / Hkv
+  FastDiv div_per_t;  // B * Hkv * pairs
+  FastDiv div_hp;     // Hkv * pairs
+  FastDiv div_pairs;  // pairs
+  FastDiv div_bh;     // B * Hkv
+  FastDiv div_hkv;    // Hkv
 };
 
 struct Item {
@@ -119,26 +148,24 @@ __device__ __forceinline__ int kv_tiles(const Params& p, int t) {
 // tiles 2t and 2t+1.
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
   Item it;
-  const int g = p.Hq / p.Hkv;
+  const int g = p.g;
   if (idx < p.items_a) {
-    const int per_t = p.B * p.Hkv * p.pairs;
-    const int tr = idx / per_t;
-    int rem = idx - tr * per_t;
+    const int tr = (int)fdiv((uint32_t)idx, p.div_per_t);
+    int rem = idx - tr * (int)p.div_per_t.d;
     const int t = p.causal ? p.nq - 1 - tr : tr;
-    it.b = rem / (p.Hkv * p.pairs);
-    rem -= it.b * p.Hkv * p.pairs;
-    it.kvh = rem / p.pairs;
+    it.b = (int)fdiv((uint32_t)rem, p.div_hp);
+    rem -= it.b * (int)p.div_hp.d;
+    it.kvh = (int)fdiv((uint32_t)rem, p.div_pairs);
     const int pp = rem - it.kvh * p.pairs;
     it.h[0] = it.kvh * g + 2 * pp;
     it.h[1] = it.h[0] + 1;
     it.t[0] = it.t[1] = t;
   } else {
     idx -= p.items_a;
-    const int per = p.B * p.Hkv;
-    const int tr = idx / per;
-    const int rem = idx - tr * per;
+    const int tr = (int)fdiv((uint32_t)idx, p.div_bh);
+    const int rem = idx - tr * (int)p.div_bh.d;
     const int tp = p.causal ? p.npq - 1 - tr : tr;
-    it.b = rem / p.Hkv;
+    it.b = (int)fdiv((uint32_t)rem, p.div_hkv);
     it.kvh = rem - it.b * p.Hkv;
     it.h[0] = it.h[1] = it.kvh * g + g - 1;
     it.t[0] = 2 * tp;
@@ -576,9 +603,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e)
             pk[e] = pack_bf16x2(__uint_as_float(ov[2 * e]) * inv_l, __uint_as_float(ov[2 * e + 1]) * inv_l);
           if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+            // 32-byte stores fill whole sectors: a warp's store touches 32 rows, and half as
+            // many such instructions keep the L1 path, which the MMAs' shared-memory operand
+            // reads also use, less busy.
+            if (p.o_align32) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+              for (int e = 0; e < 2; ++e) st_global_v8(orow + c4 * 32 + 16 * e, pk + 8 * e);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+            }
           }
         }
         if (p.lse != nullptr && in_range)

@@ -77,6 +77,18 @@ def test_bf16_small_all_elements(cuda_lib, shape):
     compare(o, lse, *_ref(x, causal), BF16_TOL, f"bf16 {shape}")
 
 
+def test_bf16_output_only_16_byte_aligned(cuda_lib):
+    # O at a 16-byte (not 32-byte) aligned address takes the 16-byte store path.
+    x = prefill_inputs(1, 4, 2, 200, 200, 128, dtype="bf16", seed=4)
+    buf = torch.zeros(x["q"].numel() + 8, dtype=torch.bfloat16, device="cuda")
+    o = buf[8:].view(x["q"].shape)
+    assert o.data_ptr() % 32 == 16
+    _, lse = attn_fwd(x["q"].cuda(), x["k"].cuda(), x["v"].cuda(), causal=True, o=o)
+    torch.cuda.synchronize()
+    compare(o, lse, *_ref(x, True), BF16_TOL, "O at 16 mod 32")
+    assert torch.all(buf[:8] == 0)
+
+
 def test_bf16_empty_keys(cuda_lib):
     x = prefill_inputs(1, 2, 1, 9, 0, 64, dtype="bf16", seed=1)
     o, lse = _run(x, False)
