@@ -49,12 +49,12 @@ constexpr int kRingStages = 5;  // K/V ring slots (with the two Q tiles: 7 x 32 
 // Register split (setmaxnreg): the launch gives every thread 168 registers (65536 / 384
 // rounded down to a multiple of 8), i.e. 64512 in total.  Warpgroup 0 (TMA, MMA, two
 // idle warps) gives registers to the two softmax warpgroups; the split per
-// head dim is the one with the fewest spills (D=128: 88 * 128 + 208 * 256 = 64512;
-// D=64: 56 * 128 + 224 * 256 = 64512).
+// head dim is the one with the fewest spills (D=128: 104 * 128 + 200 * 256 = 64512;
+// D=64: 88 * 128 + 208 * 256 = 64512).
 template <int D>
 struct Regs {
-  static constexpr int kControl = D == 128 ? 88 : 56;
-  static constexpr int kSoftmax = D == 128 ? 208 : 224;
+  static constexpr int kControl = D == 128 ? 104 : 88;
+  static constexpr int kSoftmax = D == 128 ? 200 : 208;
 };
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kFastBound = 64.0f;        // log2 units: fast-path values stay below 2^64
@@ -66,7 +66,7 @@ struct Layout {
   static constexpr int kQ = 0;              // Q[2]
   static constexpr int kRing = 2 * kTile;   // K/V ring[kRingStages]
   static constexpr int kBar = (2 + kRingStages) * kTile;
-  static constexpr int kNumBars = 2 + 2 * kRingStages + 12;
+  static constexpr int kNumBars = 4 + 2 * kRingStages + 12;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024 bytes
@@ -77,9 +77,9 @@ struct Layout {
 
 // barrier indices
 enum : int {
-  kBarQFull = 0,                          // the item's Q tiles landed
-  kBarQEmpty = 1,                         // the item's S MMAs are done with the Q tiles
-  kBarFull = 2,                           // [kRingStages] TMA bytes of a ring slot landed
+  kBarQFull = 0,                          // [2] per slot: the item's Q tile landed
+  kBarQEmpty = 2,                         // [2] per slot: the item's S MMAs are done with its Q tile
+  kBarFull = 4,                           // [kRingStages] TMA bytes of a ring slot landed
   kBarEmpty = kBarFull + kRingStages,     // [kRingStages] MMAs that read the slot have completed
   kBarSFull = kBarEmpty + kRingStages,    // [2] per slot: S_i written
   kBarP0 = kBarSFull + 2,                 // [2] per slot: P_i keys 0..63 written, O_i rescaled (128 arrivals)
@@ -235,8 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto item_of = [&](int r) -> int { return r * C + ((r & 1) ? C - 1 - (int)blockIdx.x : (int)blockIdx.x); };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kBarQFull), 1);
-    mbar_init(bar(kBarQEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarQFull + s), 1);
+      mbar_init(bar(kBarQEmpty + s), 1);
+    }
     for (int s = 0; s < kRingStages; ++s) {
       mbar_init(bar(kBarFull + s), 1);
       mbar_init(bar(kBarEmpty + s), 1);
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         int fill[kRingStages];
         for (int s = 0; s < kRingStages; ++s) fill[s] = -1;
-        int qn = 0, pos = 0;
+        int qn[2] = {0, 0}, pos = 0;
         bool alive = true;
         for (int r = 0; alive; ++r) {
           const int idx = item_of(r);
@@ -285,18 +287,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const Item it = decode_item(p, idx);
           const int N = max(it.n[0], it.n[1]);
           if (N == 0) continue;
-          // Q of this item replaces the previous item's once its S MMAs are done.
-          if (qn > 0 && !mbar_wait(bar(kBarQEmpty), (qn - 1) & 1, abort_flag)) break;
-          uint32_t qbytes = 0;
-          for (int i = 0; i < 2; ++i) qbytes += it.n[i] > 0 ? (uint32_t)L::kTile : 0u;
-          mbar_arrive_expect_tx(bar(kBarQFull), qbytes);
-          for (int i = 0; i < 2; ++i) {
+          // Q_i of this item replaces the previous one once slot i's S MMAs are done with it.
+          for (int i = 0; i < 2 && alive; ++i) {
             if (it.n[i] == 0) continue;
+            if (qn[i] > 0 && !mbar_wait(bar(kBarQEmpty + i), (qn[i] - 1) & 1, abort_flag)) {
+              alive = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar(kBarQFull + i), (uint32_t)L::kTile);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sQ0 + i * L::kTile + c * L::kBox, &tmQ, bar(kBarQFull), c * 64, it.t[i] * BM,
+              tma_load_3d(sQ0 + i * L::kTile + c * L::kBox, &tmQ, bar(kBarQFull + i), c * 64, it.t[i] * BM,
                           it.b * p.Hq + it.h[i]);
+            ++qn[i];
           }
-          ++qn;
+          if (!alive) break;
           const int zkv = it.b * p.Hkv + it.kvh;
           for (int k = 0; k < 2 * N; ++k, ++pos) {
             const int s = pos % kRingStages;
@@ -315,7 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (*abort_flag) {
           // Let copies already in flight land before the CTA's shared memory is released.
           int never = 0;
-          if (qn > 0) mbar_wait(bar(kBarQFull), (qn - 1) & 1, &never, 100000000ull);
+          for (int i = 0; i < 2; ++i)
+            if (qn[i] > 0) mbar_wait(bar(kBarQFull + i), (qn[i] - 1) & 1, &never, 100000000ull);
           for (int s = 0; s < kRingStages; ++s)
             if (fill[s] >= 0) mbar_wait(bar(kBarFull + s), fill[s] & 1, &never, 100000000ull);
         }
@@ -372,23 +377,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         };
         auto slot_of = [](int pos) { return pos % kRingStages; };
         auto phase_of = [](int pos) { return (uint32_t)((pos / kRingStages) & 1); };
-        int qn = 0, pos = 0;
+        int qn[2] = {0, 0};    // Q tiles consumed per slot (phases of QFull)
+        int pos = 0;           // ring position of the current item's K_0
         int gs[2] = {0, 0};    // KV steps issued per slot so far (phases of SFull, P0, P1, ODone)
         int done[2] = {0, 0};  // items per slot whose O has been produced (phases of OFree)
         bool ok = true;
-        for (int r = 0; ok; ++r) {
-          const int idx = item_of(r);
-          if (idx >= p.items) break;
-          const Item it = decode_item(p, idx);
+        // Next item with work for the MMAs at or after round rr (rr is advanced to it).
+        auto next_item = [&](int& rr, Item& out) -> bool {
+          for (;; ++rr) {
+            const int idx = item_of(rr);
+            if (idx >= p.items) return false;
+            out = decode_item(p, idx);
+            if (out.n[0] > 0 || out.n[1] > 0) return true;
+          }
+        };
+        int r = 0;
+        Item it;
+        bool have = next_item(r, it);
+        bool started = false;  // S_i(0) of the current item was issued by the previous item's last step
+        while (ok && have) {
           const int N = max(it.n[0], it.n[1]);
-          if (N == 0) continue;
-          if (!(ok = warp_wait(bar(kBarQFull), qn & 1, abort_flag))) break;
-          if (!(ok = warp_wait(bar(kBarFull + slot_of(pos)), phase_of(pos), abort_flag))) break;
-          // S_i(0) reuses the TMEM of the previous item's P_i: in issue order behind its PV.
-          for (int i = 0; i < 2; ++i)
-            if (it.n[i] > 0) issue_s(i, slot_of(pos));
-          commit(kBarEmpty + slot_of(pos));
-          if (N == 1) commit(kBarQEmpty);
+          int r2 = r + 1;
+          Item nx;
+          const bool have_next = next_item(r2, nx);
+          // When both slots end this item at the same step and both have work in the next one,
+          // the next item's S_i(0) follows PV_i of this item's last step like any S_i(j+1):
+          // the slots stay staggered and the tensor pipe runs on while each slot's epilogue
+          // executes.  Otherwise the next item starts with both S MMAs together.
+          const bool chain = have_next && it.n[0] == it.n[1] && nx.n[0] > 0 && nx.n[1] > 0;
+          const int pnext = pos + 2 * N;  // ring position of the next item's K_0
+          if (!started) {
+            for (int i = 0; i < 2 && ok; ++i)
+              if (it.n[i] > 0) ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag);
+            if (!ok) break;
+            if (!(ok = warp_wait(bar(kBarFull + slot_of(pos)), phase_of(pos), abort_flag))) break;
+            // S_i(0) reuses the TMEM of the previous item's P_i: in issue order behind its PV.
+            for (int i = 0; i < 2; ++i)
+              if (it.n[i] > 0) {
+                issue_s(i, slot_of(pos));
+                if (it.n[i] == 1) commit(kBarQEmpty + i);
+              }
+            commit(kBarEmpty + slot_of(pos));
+          }
           for (int j = 0; ok && j < N; ++j) {
             const int kv = pos + 2 * j + 1, kn = pos + 2 * j + 2;  // ring positions of V_j and K_{j+1}
             const int last = j < it.n[1] ? 1 : 0;                 // the last slot that multiplies by V_j
@@ -407,24 +437,30 @@ __global__ void __launch_bounds__(kThreads, 1)
               issue_pv(i, slot_of(kv), j, 4);
               commit(kBarODone + i);
               if (i == last) commit(kBarEmpty + slot_of(kv));  // V_j's slot, once its PVs are done
-              if (j + 1 < ni) {
+              if (j + 1 < ni || chain) {
+                // K_{j+1} of this item, or K_0 of the next (ring position kn == pnext then)
                 if (!next_k) {
                   if (!(ok = warp_wait(bar(kBarFull + slot_of(kn)), phase_of(kn), abort_flag))) break;
                   next_k = true;
                 }
+                if (j + 1 == ni && !(ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag))) break;
                 issue_s(i, slot_of(kn));
+                const int left = (j + 1 < ni) ? ni - (j + 1) : (i ? nx.n[1] : nx.n[0]);
+                if (left == 1) commit(kBarQEmpty + i);  // the last S MMA that reads this Q_i
               }
             }
             if (!ok) break;
-            if (j + 1 < N) commit(kBarEmpty + slot_of(kn));
-            if (j + 2 == N) commit(kBarQEmpty);  // every S MMA of the item has been issued
+            if (j + 1 < N || chain) commit(kBarEmpty + slot_of(kn));
           }
           for (int i = 0; i < 2; ++i) {
             gs[i] += it.n[i];
             done[i] += it.n[i] > 0 ? 1 : 0;
           }
-          pos += 2 * N;
-          ++qn;
+          pos = pnext;
+          started = chain;
+          it = nx;
+          r = r2;
+          have = have_next;
         }
         if (!ok) {
           int never = 0;
