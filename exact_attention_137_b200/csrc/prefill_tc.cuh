@@ -504,12 +504,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kv0 = j * BN;
         // Mask only tiles that reach past the last key or the causal diagonal.
         const bool masked = (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk;
+        // Keys 0..cl of a 32-key chunk are visible to this row: one 32-bit compare against a
+        // constant per key.
         auto mask_chunk = [&](uint32_t(&v)[32], int q4) {
+          const long long lim = (key_limit < (long long)p.Sk - 1 ? key_limit : (long long)p.Sk - 1) - kv0 - q4 * 32;
+          const int cl = (int)(lim < -1 ? -1 : (lim > 32 ? 32 : lim));
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int key = kv0 + q4 * 32 + e;
-            if ((long long)key > key_limit || key >= p.Sk) v[e] = __float_as_uint(-INFINITY);
-          }
+          for (int e = 0; e < 32; ++e) v[e] = e > cl ? __float_as_uint(-INFINITY) : v[e];
         };
         auto publish = [&](const uint32_t(&w)[32], uint32_t col, uint32_t b) {
           tmem_st32(tS + col, w);
