@@ -29,6 +29,12 @@ Readings where the pages are silent or garbled:
 4. The log-sum-exp is not on the pages.  ``LSE_i = ln sum_j exp(scale * q_i . k_j)``
    over allowed ``j`` (natural log of the *scaled* scores).
 5. ``scale`` is explicit; ``None`` means ``1/sqrt(D)`` (CSDN §五 default).
+6. Sliding-window attention is named on the CSDN page (追问4, among the long-context
+   KV-cache optimisations) but not defined.  With a window ``W >= 1`` a query at
+   absolute position ``p = i + Sk - Sq`` attends to keys ``p - W < j <= p``: causal,
+   bottom-right aligned as in reading 2, and ``W`` keys including its own.  A decode
+   step (``p = seqlen - 1``) therefore attends to the last ``W`` cached tokens.
+   ``W <= 0`` means no window.
 """
 
 from __future__ import annotations
@@ -56,13 +62,19 @@ def _default_scale(d: int, scale):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def allowed_mask(sq: int, sk: int, causal: bool, rows=None) -> np.ndarray:
-    """Boolean ``[len(rows), sk]``: may query row ``i`` attend to key ``j``? (reading 2)."""
+def allowed_mask(sq: int, sk: int, causal: bool, rows=None, window: int = 0) -> np.ndarray:
+    """Boolean ``[len(rows), sk]``: may query row ``i`` attend to key ``j``? (readings 2, 6)."""
     rows = np.arange(sq) if rows is None else np.asarray(rows, dtype=np.int64)
     cols = np.arange(sk)
     if not causal:
+        if window > 0:
+            raise ValueError("a sliding window is defined for causal attention only")
         return np.ones((rows.size, sk), dtype=bool)
-    return cols[None, :] <= (rows[:, None] + (sk - sq))
+    pos = rows[:, None] + (sk - sq)  # absolute position of the query
+    allowed = cols[None, :] <= pos
+    if window > 0:
+        allowed &= cols[None, :] > pos - window
+    return allowed
 
 
 def _softmax_times_v(s: np.ndarray, allowed: np.ndarray, v: np.ndarray):
@@ -92,7 +104,7 @@ def _check_heads(hq: int, hkv: int) -> int:
     return hq // hkv
 
 
-def attention_rows_ref(q, k, v, causal: bool = False, scale=None, rows=None):
+def attention_rows_ref(q, k, v, causal: bool = False, scale=None, rows=None, window: int = 0):
     """Exact attention for a subset of query rows (all rows when ``rows is None``).
 
     ``q``: ``[B, Hq, Sq, D]``; ``k``, ``v``: ``[B, Hkv, Sk, D]``.  Returns
@@ -109,7 +121,7 @@ def attention_rows_ref(q, k, v, causal: bool = False, scale=None, rows=None):
     # CSDN §五: ``k = np.repeat(k, group_size, axis=1)`` -- query head h reads K/V head h // g.
     k_rep = np.repeat(k, g, axis=1)
     v_rep = np.repeat(v, g, axis=1)
-    allowed = allowed_mask(sq, sk, causal, rows)
+    allowed = allowed_mask(sq, sk, causal, rows, window)
     o = np.zeros((b_, hq, rows.size, dv))
     lse = np.zeros((b_, hq, rows.size))
     for b in range(b_):
@@ -119,9 +131,9 @@ def attention_rows_ref(q, k, v, causal: bool = False, scale=None, rows=None):
     return o, lse
 
 
-def attention_ref(q, k, v, causal: bool = False, scale=None):
+def attention_ref(q, k, v, causal: bool = False, scale=None, window: int = 0):
     """Exact GQA attention, all rows: ``O [B, Hq, Sq, D]``, ``LSE [B, Hq, Sq]``."""
-    return attention_rows_ref(q, k, v, causal=causal, scale=scale, rows=None)
+    return attention_rows_ref(q, k, v, causal=causal, scale=scale, rows=None, window=window)
 
 
 def flash_blockwise_ref(q, k, v, block_q: int, block_kv: int, scale=None):
@@ -163,7 +175,7 @@ def flash_blockwise_ref(q, k, v, block_q: int, block_kv: int, scale=None):
     return out, lse
 
 
-def brute_force_attention(q, k, v, causal: bool = False, scale=None):
+def brute_force_attention(q, k, v, causal: bool = False, scale=None, window: int = 0):
     """Scalar-loop attention for tiny inputs (nested lists in, nested lists out).
 
     Independent of the NumPy path: every score, exponential and sum is a Python
@@ -187,7 +199,8 @@ def brute_force_attention(q, k, v, causal: bool = False, scale=None):
             kvh = h // g
             oh, lh = [], []
             for i in range(sq):
-                keys = [j for j in range(sk) if (not causal) or j <= i + sk - sq]
+                p = i + sk - sq
+                keys = [j for j in range(sk) if (not causal) or (j <= p and (window <= 0 or j > p - window))]
                 if not keys:
                     oh.append([0.0] * len(v[b][kvh][0]))
                     lh.append(-math.inf)
@@ -206,7 +219,7 @@ def brute_force_attention(q, k, v, causal: bool = False, scale=None):
     return out, lse
 
 
-def decode_ref(q, k_cache, v_cache, seqlens, block_table=None, block_size=None, scale=None):
+def decode_ref(q, k_cache, v_cache, seqlens, block_table=None, block_size=None, scale=None, window: int = 0):
     """One query token per sequence against its cached keys/values.
 
     ``q``: ``[B, Hq, D]``.  Contiguous cache (``block_table is None``):
@@ -216,8 +229,9 @@ def decode_ref(q, k_cache, v_cache, seqlens, block_table=None, block_size=None, 
     ``block_table[b][t // block_size]`` at slot ``t % block_size`` (gocoding §5 page
     table).  The gather is a host loop over the page table; the new token attends
     to every cached token (CSDN §七), so no causal mask applies.  ``seqlens[b]``
-    counts the cached tokens including the current one.  Returns ``O [B, Hq, D]``
-    and ``LSE [B, Hq]``.
+    counts the cached tokens including the current one.  With ``window >= 1`` only the
+    last ``window`` of them are attended to (reading 6).  Returns ``O [B, Hq, D]`` and
+    ``LSE [B, Hq]``.
     """
     q = _f64(q)
     bsz, hq, d = q.shape
@@ -243,9 +257,12 @@ def decode_ref(q, k_cache, v_cache, seqlens, block_table=None, block_size=None, 
                 cnt = min(bs, n - i * bs)
                 kb[:, i * bs : i * bs + cnt] = k_cache[blk, :, :cnt]
                 vb[:, i * bs : i * bs + cnt] = v_cache[blk, :, :cnt]
+        visible = np.ones((1, n), dtype=bool)
+        if window > 0:
+            visible[0, : max(0, n - window)] = False
         for h in range(hq):
             s = (kb[h // g] @ q[b, h]) * sc
-            o, l = _softmax_times_v(s[None, :], np.ones((1, n), dtype=bool), vb[h // g])
+            o, l = _softmax_times_v(s[None, :], visible, vb[h // g])
             out[b, h] = o[0]
             lse[b, h] = l[0]
     return out, lse

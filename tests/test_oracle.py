@@ -359,10 +359,10 @@ def test_decode_empty_sequence():
 # ---------------------------------------------------------------- planted mistakes
 
 
-def _mismatch_vs_brute(causal=True, sq=5, sk=7, scale=0.6):
+def _mismatch_vs_brute(causal=True, sq=5, sk=7, scale=0.6, window=0):
     q, k, v = _rand((1, 4, sq, 3), 80), _rand((1, 2, sk, 3), 81), _rand((1, 2, sk, 3), 82)
-    o, _ = attention_ref(q, k, v, causal=causal, scale=scale)
-    ob, _ = _bf((q, k, v, dict(causal=causal, scale=scale)))
+    o, _ = attention_ref(q, k, v, causal=causal, scale=scale, window=window)
+    ob, _ = _bf((q, k, v, dict(causal=causal, scale=scale, window=window)))
     return float(np.nanmax(np.abs(o - np.array(ob))))
 
 
@@ -379,12 +379,76 @@ def test_planted_dropped_scale_is_caught(monkeypatch):
 
 
 def test_planted_top_left_causal_is_caught(monkeypatch):
-    def top_left(sq, sk, causal, rows=None):
+    def top_left(sq, sk, causal, rows=None, window=0):
         rows = np.arange(sq) if rows is None else np.asarray(rows)
         return np.arange(sk)[None, :] <= rows[:, None] if causal else np.ones((rows.size, sk), bool)
 
     monkeypatch.setattr(oatt, "allowed_mask", top_left)
     assert _mismatch_vs_brute(sq=5, sk=7) > 1e-3
+
+
+def test_planted_window_off_by_one_is_caught(monkeypatch):
+    real = oatt.allowed_mask
+
+    def wide(sq, sk, causal, rows=None, window=0):
+        return real(sq, sk, causal, rows, window + 1 if window > 0 else 0)  # one key too many
+
+    monkeypatch.setattr(oatt, "allowed_mask", wide)
+    assert _mismatch_vs_brute(sq=6, sk=9, window=3) > 1e-3
+
+
+# ---------------------------------------------------------------- sliding window (reading 6)
+
+
+@pytest.mark.parametrize("window", [1, 2, 3, 5])
+@pytest.mark.parametrize("sq,sk", [(6, 6), (4, 9), (9, 4)])
+def test_window_matches_brute_force(window, sq, sk):
+    q, k, v = _rand((1, 4, sq, 3), 90 + window), _rand((1, 2, sk, 3), 91), _rand((1, 2, sk, 3), 92)
+    o, lse = attention_ref(q, k, v, causal=True, scale=0.7, window=window)
+    ob, lb = _bf((q, k, v, dict(causal=True, scale=0.7, window=window)))
+    ob, lb = np.array(ob), np.array(lb)
+    assert np.array_equal(np.isneginf(lse), np.isneginf(lb))
+    fin = np.isfinite(lb)
+    assert np.max(np.abs(o - ob)) < 1e-12 and np.max(np.abs(lse[fin] - lb[fin])) < 1e-12
+
+
+def test_window_covering_every_key_is_plain_causal():
+    q, k, v = _rand((2, 4, 20, 8), 95), _rand((2, 2, 24, 8), 96), _rand((2, 2, 24, 8), 97)
+    o, lse = attention_ref(q, k, v, causal=True)
+    ow, lw = attention_ref(q, k, v, causal=True, window=24)
+    assert np.array_equal(o, ow) and np.array_equal(lse, lw)
+
+
+def test_window_one_returns_own_value_row():
+    # One visible key: weight 1, O = V[p], LSE = scale * q . k_p (p = i + Sk - Sq).
+    q, k, v = _rand((1, 2, 5, 4), 98), _rand((1, 2, 8, 4), 99), _rand((1, 2, 8, 4), 100)
+    o, lse = attention_ref(q, k, v, causal=True, scale=0.5, window=1)
+    for h in range(2):
+        for i in range(5):
+            p = i + 3
+            assert np.array_equal(o[0, h, i], v[0, h, p])
+            assert abs(lse[0, h, i] - 0.5 * float(q[0, h, i] @ k[0, h, p])) < 1e-12
+
+
+def test_window_ignores_keys_outside_it():
+    # Keys and values at or before p - W never reach row p: changing them changes nothing.
+    q, k, v = _rand((1, 2, 16, 8), 101), _rand((1, 1, 16, 8), 102), _rand((1, 1, 16, 8), 103)
+    W, i = 4, 12
+    o, lse = attention_rows_ref(q, k, v, causal=True, rows=[i], window=W)
+    k2, v2 = k.copy(), v.copy()
+    k2[:, :, : i - W + 1] = 50.0
+    v2[:, :, : i - W + 1] = -7.0
+    o2, lse2 = attention_rows_ref(q, k2, v2, causal=True, rows=[i], window=W)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_window_decode_is_last_windowed_row():
+    rng = np.random.Generator(np.random.PCG64(104))
+    n, W = 37, 10
+    q, k, v = rng.standard_normal((1, 4, n, 16)), rng.standard_normal((1, 2, n, 16)), rng.standard_normal((1, 2, n, 16))
+    o, lse = attention_rows_ref(q, k, v, causal=True, rows=[n - 1], window=W)
+    od, ld = decode_ref(q[:, :, n - 1], k, v, np.array([n]), window=W)
+    assert np.max(np.abs(od - o[:, :, 0])) < 1e-12 and np.max(np.abs(ld - lse[:, :, 0])) < 1e-12
 
 
 # ---------------------------------------------------------------- plan restatement
