@@ -45,6 +45,10 @@ _SIGS = {
                           _c_int, _c_int, _vp]),
     "attn_decode": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                              _c_int, _c_float, _vp, _size_t, _vp, _vp, _c_int, _vp]),
+    "attn_fwd_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_float,
+                                 _c_int, _c_int, _vp]),
+    "attn_decode_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                    _c_int, _c_float, _c_int, _vp, _size_t, _vp, _vp, _c_int, _vp]),
     "attn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_int, _c_float, _vp, _vp, _c_int, _vp]),
     "attn_decode_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
@@ -122,11 +126,12 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, lse=None,
-             return_lse: bool = True, stream=None):
+             return_lse: bool = True, stream=None, window: int | None = None):
     """Attention forward: ``q [B,Hq,Sq,D]``, ``k``/``v`` ``[B,Hkv,Sk,D]`` on the GPU.
 
-    Returns ``(o, lse)`` (``lse`` is ``None`` when ``return_lse`` is false and none
-    was passed).
+    ``window`` (causal only) selects ``attn_fwd_window``: each query sees its last
+    ``window`` keys.  Returns ``(o, lse)`` (``lse`` is ``None`` when ``return_lse`` is
+    false and none was passed).
     """
     lib = load()
     if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
@@ -147,6 +152,13 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
     if lse is None and return_lse:
         lse = torch.empty((B, Hq, Sq), device=q.device, dtype=torch.float32)
     sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if window is not None:
+        if not causal:
+            raise ValueError("a sliding window needs causal=True")
+        st = lib.attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, sc,
+                                 int(window), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+        _check(st, "attn_fwd_window")
+        return o, lse
     st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Sk, D, sc,
                       1 if causal else 0, _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
     _check(st, "attn_fwd")
@@ -189,12 +201,13 @@ def decode_workspace(B, Hq, Hkv, D, max_seqlen, device) -> torch.Tensor:
 
 def attn_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None, block_size: int | None = None,
                 scale: float | None = None, workspace=None, o=None, lse=None, return_lse: bool = True,
-                stream=None):
+                stream=None, window: int | None = None):
     """Single-token decode.  ``q [B,Hq,D]`` bf16; ``seqlens [B]`` int32 on the GPU.
 
     Paged: ``k_cache``/``v_cache`` ``[num_blocks,Hkv,block_size,D]`` and
     ``block_table [B,max_blocks]`` int32.  Contiguous: ``[B,Hkv,cap,D]`` and
-    ``block_table=None``.  Returns ``(o, lse)``.
+    ``block_table=None``.  ``window`` selects ``attn_decode_window`` (the last
+    ``window`` tokens only).  Returns ``(o, lse)``.
     """
     lib = load()
     if q.dim() != 3:
@@ -229,6 +242,13 @@ def attn_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None,
     if lse is None and return_lse:
         lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
     sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    if window is not None:
+        st = lib.attn_decode_window(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(block_table), bs,
+                                    max_blocks, num_blocks, int(max_seqlen), B, Hq, Hkv, D, sc, int(window),
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(o),
+                                    _ptr(lse), _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
+        _check(st, "attn_decode_window")
+        return o, lse
     st = lib.attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(block_table), bs, max_blocks,
                          num_blocks, int(max_seqlen), B, Hq, Hkv, D, sc, _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _ptr(o), _ptr(lse), _dtype_code(q),

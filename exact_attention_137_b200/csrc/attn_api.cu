@@ -99,7 +99,7 @@ int device_sms() {
 
 template <int D>
 int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Sq, int Sk, float scale, int causal, cudaStream_t st) {
+                  int Hkv, int Sq, int Sk, float scale, int causal, int window, cudaStream_t st) {
   using Lay = attn::tc::Layout<D>;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_bf16(&tq, q, D, Sq, (long long)B * Hq) || !make_tmap_bf16(&tk, k, D, Sk, (long long)B * Hkv) ||
@@ -115,6 +115,7 @@ int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* l
   p.Sk = Sk;
   p.scale_log2 = scale * attn::kLog2e;
   p.causal = causal ? 1 : 0;
+  p.window = causal ? window : 0;
   p.nq = (int)cdiv(Sq, BM);
   const int g = Hq / Hkv;
   p.pairs = g / 2;
@@ -144,12 +145,12 @@ int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* l
 
 template <typename T, int D>
 int launch_fwd_simt(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                    int Hkv, int Sq, int Sk, float scale, int causal, cudaStream_t st) {
+                    int Hkv, int Sq, int Sk, float scale, int causal, int window, cudaStream_t st) {
   dim3 grid((unsigned)cdiv(Sq, attn::simt::kRowsPerBlock), (unsigned)(B * Hq));
   if (grid.y > 65535u) return ATTN_ERR_UNSUPPORTED;
   attn::simt::fwd_simt_kernel<T, D><<<grid, attn::simt::kRowsPerBlock * 32, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o), lse,
-      Hq, Hkv, Sq, Sk, scale * attn::kLog2e, causal ? 1 : 0);
+      Hq, Hkv, Sq, Sk, scale * attn::kLog2e, causal ? 1 : 0, causal ? window : 0);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -296,11 +297,42 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   }
   if (dtype == ATTN_BF16) {
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ARG;
-    return D == 64 ? launch_fwd_tc<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st)
-                   : launch_fwd_tc<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st);
+    return D == 64 ? launch_fwd_tc<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, 0, st)
+                   : launch_fwd_tc<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, 0, st);
   }
-  return D == 64 ? launch_fwd_simt<float, 64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st)
-                 : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, st);
+  return D == 64 ? launch_fwd_simt<float, 64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, 0, st)
+                 : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, 0, st);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                    int Sq, int Sk, int D, float scale, int window, int dtype, void* stream) {
+  const int causal = 1;
+  if (window < 0) return ATTN_ERR_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || !std::isfinite(scale) || !(scale > 0.f))
+    return ATTN_ERR_ARG;
+  // q/o may be NULL only when Sq == 0, k/v only when Sk == 0 (nothing is read or written).
+  if ((Sq > 0 && (!q || !o)) || (Sk > 0 && (!k || !v))) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > INT_MAX / 2 || (long long)Sq * D > INT_MAX || (long long)Sk * D > INT_MAX)
+    return ATTN_ERR_UNSUPPORTED;
+  cudaStream_t st = as_stream(stream);
+  if (Sq == 0) return ATTN_OK;
+  const size_t elem = dtype == ATTN_BF16 ? 2 : 4;
+  if (Sk == 0) {
+    const size_t rows = (size_t)B * Hq * Sq;
+    if (cudaMemsetAsync(o, 0, rows * D * elem, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (lse) fill_empty_rows_kernel<<<(unsigned)cdiv((long long)rows, 256), 256, 0, st>>>(lse, rows);
+    return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+  if (dtype == ATTN_BF16) {
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_ARG;
+    return D == 64 ? launch_fwd_tc<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st)
+                   : launch_fwd_tc<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st);
+  }
+  return D == 64 ? launch_fwd_simt<float, 64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st)
+                 : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st);
 }
 
 int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int num_sms, int* ctas, int* heads_per_cta) {
@@ -353,10 +385,11 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen
   return ws_layout(B, D, pl).total;
 }
 
-int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
-                int block_size, int max_blocks, int num_blocks, int max_seqlen, int B, int Hq, int Hkv, int D,
-                float scale, void* workspace, size_t workspace_bytes, void* o, float* lse, int dtype,
-                void* stream) {
+int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
+                       const int* block_table, int block_size, int max_blocks, int num_blocks, int max_seqlen, int B,
+                       int Hq, int Hkv, int D, float scale, int window, void* workspace, size_t workspace_bytes,
+                       void* o, float* lse, int dtype, void* stream) {
+  if (window < 0) return ATTN_ERR_ARG;
   if (!q || !k_cache || !v_cache || !seqlens || !o) return ATTN_ERR_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || block_size <= 0 || max_seqlen < 0 || !std::isfinite(scale))
     return ATTN_ERR_ARG;
@@ -391,6 +424,7 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.nsub = (Hq / Hkv) / pl.G;
+  p.window = window;
   p.scale_log2 = scale * attn::kLog2e;
   const WsLayout wl = ws_layout(B, D, pl);
   const int sms = device_sms();
@@ -404,6 +438,14 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
   cudaStream_t st = as_stream(stream);
   const int ctas = plan_ctas(pl, sms);
   return D == 64 ? dispatch_decode_g<64>(p, pl.G, ctas, st) : dispatch_decode_g<128>(p, pl.G, ctas, st);
+}
+
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
+                int block_size, int max_blocks, int num_blocks, int max_seqlen, int B, int Hq, int Hkv, int D,
+                float scale, void* workspace, size_t workspace_bytes, void* o, float* lse, int dtype,
+                void* stream) {
+  return attn_decode_window(q, k_cache, v_cache, seqlens, block_table, block_size, max_blocks, num_blocks, max_seqlen,
+                            B, Hq, Hkv, D, scale, 0, workspace, workspace_bytes, o, lse, dtype, stream);
 }
 
 int attn_decode_check(void* workspace, void* stream) {

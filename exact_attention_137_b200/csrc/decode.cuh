@@ -165,6 +165,7 @@ struct Params {
   int block_size, max_blocks, num_blocks, max_seqlen;
   int B, Hq, Hkv;
   int nsub;  // query-head subgroups of G per KV head
+  int window;  // > 0: attend to the last `window` cached tokens only
   float scale_log2;
   float* ws_o;    // [grid][2][G][D] partial outputs per CTA slot
   float* ws_lse;  // [grid][2][G]
@@ -216,6 +217,12 @@ __device__ __forceinline__ int checked_len(const Params& p, int b, bool report) 
   return len;
 }
 
+// Tokens of sequence b that the step attends to: its length, or the last `window` of them.
+__device__ __forceinline__ int span_len(const Params& p, int b, bool report) {
+  const int len = checked_len(p, b, report);
+  return (p.window > 0 && len > p.window) ? p.window : len;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
   asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -241,7 +248,7 @@ __device__ __forceinline__ long long total_units(const Params& p, int Y, int lan
   long long sum = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
     const int b = b0 + lane;
-    sum += b < p.B ? units_of(checked_len(p, b, report)) : 0;
+    sum += b < p.B ? units_of(span_len(p, b, report)) : 0;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += shfl_ll(sum, lane ^ o);
@@ -262,7 +269,7 @@ __device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long tot
   long long prefix = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
     const int b = b0 + lane;
-    const int len = b < p.B ? checked_len(p, b, false) : 0;
+    const int len = b < p.B ? span_len(p, b, false) : 0;
     const long long span = (long long)Y * units_of(len);
     long long incl = span;
 #pragma unroll
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   }
   const int n = active_ctas(total, gridDim.x);
   if ((int)blockIdx.x >= n) return;
-  auto len_of = [&](int b) -> int { return checked_len(p, b, false); };
+  auto len_of = [&](int b) -> int { return span_len(p, b, false); };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -381,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
       auto load_id = [&](int page) -> int {
         return (paged && page < p.max_blocks) ? __ldg(table + page) : -1;
       };
-      int cur_first = sg.tok0 / bs;
+      // Segment tokens count from the first attended token; the cache holds them from `base`.
+      const int base = p.window > 0 ? checked_len(p, sg.b, false) - len_of(sg.b) : 0;
+      int cur_first = (base + sg.tok0) / bs;
       int nxt_first = cur_first + 32;
       int cur_id = load_id(cur_first + lane);
       int nxt_id = load_id(nxt_first + lane);
@@ -401,8 +410,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
                     full_bar(s));
         }
         for (int tok = a; tok < e;) {
-          const int page = tok / bs;
-          const int slot = tok - page * bs;
+          const int page = (base + tok) / bs;
+          const int slot = base + tok - page * bs;
           const int run = min(bs - slot, e - tok);
           while (page >= cur_first + 32) {
             cur_id = nxt_id;

@@ -51,7 +51,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kRowsPerBlock * 32)
     fwd_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                     T* __restrict__ o, float* __restrict__ lse, int Hq, int Hkv, int Sq, int Sk,
-                    float scale_log2, int causal) {
+                    float scale_log2, int causal, int window) {
   __shared__ float qs[kRowsPerBlock][D];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row = blockIdx.x * kRowsPerBlock + warp;
@@ -69,13 +69,15 @@ __global__ void __launch_bounds__(kRowsPerBlock * 32)
   long long last = causal ? (long long)row + Sk - Sq : (long long)Sk - 1;
   if (last > Sk - 1) last = Sk - 1;
   const int nkeys = last < 0 ? 0 : (int)last + 1;
+  // Sliding window (causal only): keys last - window + 1 .. last.
+  const int kfirst = (window > 0 && nkeys > window) ? nkeys - window : 0;
 
   float m = -INFINITY, l = 0.f;
   float acc[D / 32];
 #pragma unroll
   for (int e = 0; e < D / 32; ++e) acc[e] = 0.f;
 
-  for (int k0 = 0; k0 < nkeys; k0 += 32) {
+  for (int k0 = kfirst; k0 < nkeys; k0 += 32) {
     const int key = k0 + lane;
     float x = -INFINITY;
     if (key < nkeys) {

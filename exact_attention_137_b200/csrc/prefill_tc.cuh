@@ -117,6 +117,7 @@ struct Params {
   int B, Hq, Hkv, Sq, Sk;
   float scale_log2;  // scale * log2(e)
   int causal;
+  int window;       // > 0: causal sliding window of this many keys (0: none)
   int nq;           // query tiles per head
   int pairs;        // head pairs per KV group (g / 2)
   int items_a;      // work items made of head pairs
@@ -133,7 +134,8 @@ struct Params {
 
 struct Item {
   int b, kvh;
-  int h[2], t[2], n[2];
+  int h[2], t[2];
+  int f[2], n[2];  // per slot: first KV tile and number of KV tiles
 };
 
 __device__ __forceinline__ int kv_tiles(const Params& p, int t) {
@@ -141,6 +143,14 @@ __device__ __forceinline__ int kv_tiles(const Params& p, int t) {
   long long last = (long long)t * BM + BM - 1 + (long long)p.Sk - p.Sq;
   if (last > p.Sk - 1) last = p.Sk - 1;
   return last < 0 ? 0 : (int)(last / BN) + 1;
+}
+
+// First KV tile any row of query tile t can see: 0, or with a sliding window the tile of the
+// first row's earliest key p - W + 1 (p = row + Sk - Sq).
+__device__ __forceinline__ int kv_first(const Params& p, int t) {
+  if (p.window <= 0) return 0;
+  const long long first = (long long)t * BM + (long long)p.Sk - p.Sq - p.window + 1;
+  return first <= 0 ? 0 : (int)(first / BN);
 }
 
 // Work items, longest first under a causal mask.  Items [0, items_a): two heads of one KV
@@ -171,8 +181,34 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
     it.t[0] = 2 * tp;
     it.t[1] = 2 * tp + 1;
   }
-  for (int i = 0; i < 2; ++i) it.n[i] = it.t[i] < p.nq ? kv_tiles(p, it.t[i]) : 0;
+  for (int i = 0; i < 2; ++i) {
+    const int hi = it.t[i] < p.nq ? kv_tiles(p, it.t[i]) : 0;
+    it.f[i] = it.t[i] < p.nq ? kv_first(p, it.t[i]) : 0;
+    if (it.f[i] > hi) it.f[i] = hi;
+    it.n[i] = hi - it.f[i];
+  }
   return it;
+}
+
+// KV tiles [F, F + N) cover both slots of an item; slot i works on steps [st[i], st[i] + n[i])
+// of that range (N = 0: no MMA work).  The two ranges always overlap or touch: consecutive
+// query tiles' windows start at most one tile apart.
+struct Span {
+  int F, N, st[2];
+};
+
+__device__ __forceinline__ Span item_span(const Item& it) {
+  Span sp;
+  int lo = 0x7fffffff, hi = 0;
+  for (int i = 0; i < 2; ++i)
+    if (it.n[i] > 0) {
+      lo = min(lo, it.f[i]);
+      hi = max(hi, it.f[i] + it.n[i]);
+    }
+  sp.F = hi > 0 ? lo : 0;
+  sp.N = hi > 0 ? hi - lo : 0;
+  for (int i = 0; i < 2; ++i) sp.st[i] = it.n[i] > 0 ? it.f[i] - sp.F : 0;
+  return sp;
 }
 
 // All lanes wait; the warp proceeds only if every lane saw the phase complete.
@@ -285,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int idx = item_of(r);
           if (idx >= p.items) break;
           const Item it = decode_item(p, idx);
-          const int N = max(it.n[0], it.n[1]);
+          const Span sp = item_span(it);
+          const int N = sp.N;
           if (N == 0) continue;
           // Q_i of this item replaces the previous one once slot i's S MMAs are done with it.
           for (int i = 0; i < 2 && alive; ++i) {
@@ -312,7 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar(kBarFull + s), L::kTile);
             const void* tm = (k & 1) ? static_cast<const void*>(&tmV) : static_cast<const void*>(&tmK);
             for (int c = 0; c < D / 64; ++c)
-              tma_load_3d(sR0 + s * L::kTile + c * L::kBox, tm, bar(kBarFull + s), c * 64, (k >> 1) * BN, zkv);
+              tma_load_3d(sR0 + s * L::kTile + c * L::kBox, tm, bar(kBarFull + s), c * 64, (sp.F + (k >> 1)) * BN,
+                          zkv);
             fill[s] = f;
           }
         }
@@ -396,24 +434,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool have = next_item(r, it);
         bool started = false;  // S_i(0) of the current item was issued by the previous item's last step
         while (ok && have) {
-          const int N = max(it.n[0], it.n[1]);
+          const Span sp = item_span(it);
+          const int N = sp.N;
           int r2 = r + 1;
           Item nx;
           const bool have_next = next_item(r2, nx);
-          // When both slots end this item at the same step and both have work in the next one,
-          // the next item's S_i(0) follows PV_i of this item's last step like any S_i(j+1):
-          // the slots stay staggered and the tensor pipe runs on while each slot's epilogue
-          // executes.  Otherwise the next item starts with both S MMAs together.
-          const bool chain = have_next && it.n[0] == it.n[1] && nx.n[0] > 0 && nx.n[1] > 0;
+          // When both slots end this item at the same step and both start the next one at its
+          // first tile, the next item's S_i(0) follows PV_i of this item's last step like any
+          // S_i(j+1): the slots stay staggered and the tensor pipe runs on while each slot's
+          // epilogue executes.  Otherwise the next item starts with both S MMAs together.
+          bool chain = false;
+          if (have_next && it.n[0] > 0 && it.n[1] > 0 && nx.n[0] > 0 && nx.n[1] > 0) {
+            const Span spn = item_span(nx);
+            chain = sp.st[0] + it.n[0] == N && sp.st[1] + it.n[1] == N && spn.st[0] == 0 && spn.st[1] == 0;
+          }
           const int pnext = pos + 2 * N;  // ring position of the next item's K_0
           if (!started) {
             for (int i = 0; i < 2 && ok; ++i)
-              if (it.n[i] > 0) ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag);
+              if (it.n[i] > 0 && sp.st[i] == 0) ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag);
             if (!ok) break;
             if (!(ok = warp_wait(bar(kBarFull + slot_of(pos)), phase_of(pos), abort_flag))) break;
             // S_i(0) reuses the TMEM of the previous item's P_i: in issue order behind its PV.
             for (int i = 0; i < 2; ++i)
-              if (it.n[i] > 0) {
+              if (it.n[i] > 0 && sp.st[i] == 0) {
                 issue_s(i, slot_of(pos));
                 if (it.n[i] == 1) commit(kBarQEmpty + i);
               }
@@ -421,31 +464,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           for (int j = 0; ok && j < N; ++j) {
             const int kv = pos + 2 * j + 1, kn = pos + 2 * j + 2;  // ring positions of V_j and K_{j+1}
-            const int last = j < it.n[1] ? 1 : 0;                 // the last slot that multiplies by V_j
+            bool act[2];
+            for (int i = 0; i < 2; ++i) act[i] = it.n[i] > 0 && j >= sp.st[i] && j < sp.st[i] + it.n[i];
+            const int last = act[1] ? 1 : 0;  // the last slot that multiplies by V_j
             bool next_k = false;
             if (!(ok = warp_wait(bar(kBarFull + slot_of(kv)), phase_of(kv), abort_flag))) break;
+            if (!act[0] && !act[1]) commit(kBarEmpty + slot_of(kv));  // no slot needs V_j
             for (int i = 0; i < 2; ++i) {
-              const int ni = i ? it.n[1] : it.n[0];
-              if (j >= ni) continue;
-              const uint32_t ph = (uint32_t)((gs[i] + j) & 1);
-              if (!(ok = warp_wait(bar(kBarP0 + i), ph, abort_flag))) break;
-              // PV_i(0) overwrites O_i: the previous item's epilogue must have read it.
-              if (j == 0 && done[i] > 0 && !(ok = warp_wait(bar(kBarOFree + i), (done[i] - 1) & 1, abort_flag)))
-                break;
-              issue_pv(i, slot_of(kv), j, 0);
-              if (!(ok = warp_wait(bar(kBarP1 + i), ph, abort_flag))) break;
-              issue_pv(i, slot_of(kv), j, 4);
-              commit(kBarODone + i);
-              if (i == last) commit(kBarEmpty + slot_of(kv));  // V_j's slot, once its PVs are done
-              if (j + 1 < ni || chain) {
+              const int ni = it.n[i], s0 = sp.st[i];
+              if (act[i]) {
+                const int jj = j - s0;  // the slot's own step
+                const uint32_t ph = (uint32_t)((gs[i] + jj) & 1);
+                if (!(ok = warp_wait(bar(kBarP0 + i), ph, abort_flag))) break;
+                // PV_i(0) overwrites O_i: the previous item's epilogue must have read it.
+                if (jj == 0 && done[i] > 0 && !(ok = warp_wait(bar(kBarOFree + i), (done[i] - 1) & 1, abort_flag)))
+                  break;
+                issue_pv(i, slot_of(kv), jj, 0);
+                if (!(ok = warp_wait(bar(kBarP1 + i), ph, abort_flag))) break;
+                issue_pv(i, slot_of(kv), jj, 4);
+                commit(kBarODone + i);
+                if (i == last) commit(kBarEmpty + slot_of(kv));  // V_j's slot, once its PVs are done
+              }
+              const bool act_next = ni > 0 && j + 1 >= s0 && j + 1 < s0 + ni;
+              const bool into_next = chain && j == N - 1;
+              if (act_next || into_next) {
                 // K_{j+1} of this item, or K_0 of the next (ring position kn == pnext then)
                 if (!next_k) {
                   if (!(ok = warp_wait(bar(kBarFull + slot_of(kn)), phase_of(kn), abort_flag))) break;
                   next_k = true;
                 }
-                if (j + 1 == ni && !(ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag))) break;
+                // The slot's first S of an item reads a new Q_i.
+                if ((into_next || j + 1 == s0) && !(ok = warp_wait(bar(kBarQFull + i), qn[i]++ & 1, abort_flag)))
+                  break;
                 issue_s(i, slot_of(kn));
-                const int left = (j + 1 < ni) ? ni - (j + 1) : (i ? nx.n[1] : nx.n[0]);
+                const int left = into_next ? nx.n[i] : s0 + ni - (j + 1);
                 if (left == 1) commit(kBarQEmpty + i);  // the last S MMA that reads this Q_i
               }
             }
@@ -487,12 +539,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (idx >= p.items) break;
       const Item it = decode_item(p, idx);
       const int n = i ? it.n[1] : it.n[0];
+      const int f = i ? it.f[1] : it.f[0];  // first KV tile
       const int t = i ? it.t[1] : it.t[0];
       const int h = i ? it.h[1] : it.h[0];
       if (t >= p.nq) continue;  // this slot has no query tile in the item
       const int qrow = t * BM + row;
       const long long key_limit = p.causal ? (long long)qrow + p.Sk - p.Sq : (long long)p.Sk - 1;
       const long long tile_limit = p.causal ? (long long)t * BM + p.Sk - p.Sq : (long long)p.Sk - 1;
+      // Sliding window: this row's first visible key, and the largest first key of the tile's rows.
+      const long long key_first = p.window > 0 ? (long long)qrow + p.Sk - p.Sq - p.window + 1 : 0;
+      const long long tile_first = p.window > 0 ? (long long)t * BM + BM - 1 + p.Sk - p.Sq - p.window + 1 : 0;
       const float c = p.scale_log2;
       const uint64_t c2 = f2pack(c, c);
       // l: fp32 row sum (for the LSE); lr: row sum of the bf16 P that the tensor core
@@ -501,16 +557,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; j < n; ++j) {
         if (!(ok = warp_wait(bar_s, (gs + j) & 1, abort_flag))) break;
         tc_fence_after();
-        const int kv0 = j * BN;
-        // Mask only tiles that reach past the last key or the causal diagonal.
-        const bool masked = (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk;
-        // Keys 0..cl of a 32-key chunk are visible to this row: one 32-bit compare against a
-        // constant per key.
+        const int kv0 = (f + j) * BN;
+        // Mask only tiles that reach past the last key or the causal diagonal, or (window) start
+        // before some row's first key.
+        const bool masked = (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk || (long long)kv0 < tile_first;
+        // Keys lo..hi of a 32-key chunk are visible to this row: compares against constants.
         auto mask_chunk = [&](uint32_t(&v)[32], int q4) {
           const long long lim = (key_limit < (long long)p.Sk - 1 ? key_limit : (long long)p.Sk - 1) - kv0 - q4 * 32;
           const int cl = (int)(lim < -1 ? -1 : (lim > 32 ? 32 : lim));
+          const long long flo = key_first - kv0 - q4 * 32;
+          const int cf = (int)(flo < 0 ? 0 : (flo > 33 ? 33 : flo));
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = e > cl ? __float_as_uint(-INFINITY) : v[e];
+          for (int e = 0; e < 32; ++e) v[e] = (e > cl || e < cf) ? __float_as_uint(-INFINITY) : v[e];
         };
         auto publish = [&](const uint32_t(&w)[32], uint32_t col, uint32_t b) {
           tmem_st32(tS + col, w);

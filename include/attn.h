@@ -77,6 +77,17 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal,
              int dtype, void* stream);
 
+/* attn_fwd_window: causal prefill with a sliding window (CSDN «注意力变体深挖», 追问4,
+ * names sliding-window attention among the long-context optimisations without defining
+ * it).  Query row i, at absolute position p = i + Sk - Sq, attends to the keys
+ * p - window < j <= p: the causal mask of attn_fwd, restricted to the last `window` keys
+ * including its own.  window == 0 is plain causal attention; window >= Sk changes nothing.
+ * KV tiles that no row of a query tile can see are not read.  Arguments, layouts and
+ * tolerances as attn_fwd.  Returns ATTN_ERR_ARG for window < 0, else as attn_fwd. */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int window,
+                    int dtype, void* stream);
+
 /* ------------------------------------------------------------------ decode
  * Single-token decode against a KV cache (CSDN «注意力变体深挖» §七: each step
  * computes only the new token's Q against the cached K/V; gocoding §5: a paged cache
@@ -121,6 +132,19 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache,
                 int B, int Hq, int Hkv, int D, float scale,
                 void* workspace, size_t workspace_bytes,
                 void* o, float* lse, int dtype, void* stream);
+
+/* attn_decode_window: attn_decode with a sliding window (same reading as attn_fwd_window):
+ * the new token, at position seqlens[b] - 1, attends to the last `window` cached tokens
+ * of its sequence only (all of them when seqlens[b] <= window); the others are not read.
+ * window == 0 is attn_decode.  The split schedule is that of attn_decode with every
+ * length replaced by min(seqlens[b], window).  Returns ATTN_ERR_ARG for window < 0, else
+ * as attn_decode. */
+int attn_decode_window(const void* q, const void* k_cache, const void* v_cache,
+                       const int* seqlens, const int* block_table,
+                       int block_size, int max_blocks, int num_blocks, int max_seqlen,
+                       int B, int Hq, int Hkv, int D, float scale, int window,
+                       void* workspace, size_t workspace_bytes,
+                       void* o, float* lse, int dtype, void* stream);
 
 /* attn_decode_noalloc: the same decode as attn_decode, for callers that cannot allocate
  * device memory at all -- for example code running inside an allocator callback, a

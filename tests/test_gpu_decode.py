@@ -158,3 +158,40 @@ def test_bounded_wait_reports_timeout(cuda_lib):
     x = decode_contiguous_inputs(1, 4, 1, 64, 32, 0, 0, seed=7, seqlens=[32])
     o, lse = _run(x)
     compare(o, lse, *_ref(x), BF16_TOL, "after timeout")
+
+
+# ---------------------------------------------------------------- sliding window
+
+
+@pytest.mark.parametrize("case", [
+    # kind, B, Hq, Hkv, D, lengths, window, block size
+    ("contiguous", 4, 32, 8, 128, [1000, 33, 64, 1099], 100, None),
+    ("contiguous", 3, 8, 8, 64, [500, 1, 257], 1, None),
+    ("paged", 4, 32, 8, 128, [512, 8192, 77, 3000], 1000, 16),
+    ("paged", 2, 16, 4, 64, [23, 101], 37, 5),
+    ("paged", 2, 32, 1, 128, [700, 129], 130, 16),   # MQA
+])
+def test_window(cuda_lib, case):
+    kind, B, Hq, Hkv, D, lens, W, bs = case
+    if kind == "contiguous":
+        x = decode_contiguous_inputs(B, Hq, Hkv, D, max(lens), 0, 0, seed=W, seqlens=lens)
+    else:
+        x = decode_paged_inputs(B, Hq, Hkv, D, bs, 0, max(lens), seed=W, seqlens=lens, extra_blocks=2)
+    g = _gpu(x)
+    o, lse = attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=g["max_seqlen"],
+                         block_table=g["block_table"], block_size=g["block_size"], window=W)
+    torch.cuda.synchronize()
+    bt = None if x["block_table"] is None else x["block_table"].numpy()
+    ref = decode_ref(to_f64(x["q"]), x["k_cache"].float().numpy(), x["v_cache"].float().numpy(), x["seqlens"].numpy(),
+                     block_table=bt, block_size=x["block_size"], window=W)
+    compare(o, lse, *ref, BF16_TOL, f"window {case[:2]} W={W}")
+
+
+def test_window_longer_than_every_sequence_is_plain_decode(cuda_lib):
+    x = decode_paged_inputs(3, 32, 8, 128, 16, 0, 900, seed=5, seqlens=[900, 17, 300])
+    g = _gpu(x)
+    o1, l1 = _run(x)
+    o2, l2 = attn_decode(g["q"], g["k_cache"], g["v_cache"], g["seqlens"], max_seqlen=g["max_seqlen"],
+                         block_table=g["block_table"], block_size=g["block_size"], window=900)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

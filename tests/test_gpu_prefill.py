@@ -13,7 +13,7 @@ import pytest
 import torch
 
 from oracle import attention_ref, attention_rows_ref
-from exact_attention_137_b200 import attn_fwd, device_status
+from exact_attention_137_b200 import _lib, attn_fwd, device_status
 from exact_attention_137_b200.workloads import prefill_inputs, to_f64
 
 from parity import BF16_TOL, F32_TOL, compare
@@ -159,3 +159,66 @@ def test_polynomial_exp2_against_exp2(cuda_lib):
     # below the clamp: tiny, positive, finite
     z = _lib.selftest_exp2_poly(torch.tensor([-200.0, -1e30, -127.5], device="cuda")).cpu()
     assert torch.all(z >= 0) and torch.all(z < 1e-37)
+
+
+# ---------------------------------------------------------------- sliding window
+
+
+WINDOW_SHAPES = [
+    # B, Hq, Hkv, Sq, Sk, D, window
+    (1, 4, 2, 520, 520, 128, 200),    # head pairs, window not a multiple of the tile
+    (1, 3, 3, 700, 700, 128, 128),    # MHA: the two query tiles of an item start at different KV tiles
+    (1, 6, 2, 640, 640, 128, 300),    # g = 3: head pair plus leftover head
+    (2, 8, 1, 300, 450, 64, 50),      # Sq < Sk, D = 64
+    (1, 4, 2, 384, 256, 128, 64),     # Sq > Sk: fully masked leading rows
+    (1, 2, 1, 260, 260, 128, 1),      # each row sees only its own key
+]
+
+
+@pytest.mark.parametrize("shape", WINDOW_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_bf16_window_all_elements(cuda_lib, shape):
+    B, Hq, Hkv, Sq, Sk, D, W = shape
+    x = prefill_inputs(B, Hq, Hkv, Sq, Sk, D, dtype="bf16", seed=sum(shape))
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = attn_fwd(q, k, v, causal=True, window=W)
+    torch.cuda.synchronize()
+    ref = attention_rows_ref(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), causal=True, window=W)
+    compare(o, lse, *ref, BF16_TOL, f"window {shape}")
+
+
+def test_window_covering_all_keys_is_causal_bit_for_bit(cuda_lib):
+    x = prefill_inputs(1, 4, 2, 600, 600, 128, dtype="bf16", seed=11)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o1, l1 = attn_fwd(q, k, v, causal=True)
+    o2, l2 = attn_fwd(q, k, v, causal=True, window=600)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fp32_window(cuda_lib):
+    x = prefill_inputs(1, 4, 2, 200, 200, 64, dtype="f32", seed=12)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = attn_fwd(q, k, v, causal=True, window=33)
+    torch.cuda.synchronize()
+    compare(o, lse, *attention_rows_ref(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), causal=True, window=33),
+            F32_TOL, "fp32 window")
+
+
+@pytest.mark.parametrize("hkv", [8, 32])
+def test_window_4k_sampled(cuda_lib, hkv):
+    x = prefill_inputs(1, 32, hkv, 4096, 4096, 128, dtype="bf16", seed=13)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o, lse = attn_fwd(q, k, v, causal=True, window=1000)
+    torch.cuda.synchronize()
+    rows = _sample_rows(4096, 160, seed=hkv, must=(999, 1000, 1001, 2047, 2048))
+    ref = attention_rows_ref(to_f64(x["q"]), to_f64(x["k"]), to_f64(x["v"]), causal=True, rows=rows, window=1000)
+    compare(o[:, :, rows], lse[:, :, rows], *ref, BF16_TOL, f"window 4k Hkv={hkv}")
+
+
+def test_window_rejects_negative_and_non_causal(cuda_lib):
+    x = prefill_inputs(1, 2, 1, 16, 16, 64, dtype="bf16", seed=14)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    with pytest.raises(_lib.AttnError):
+        attn_fwd(q, k, v, causal=True, window=-1)
+    with pytest.raises(ValueError):
+        attn_fwd(q, k, v, causal=False, window=4)
