@@ -14,6 +14,9 @@ Recipe (every draw is seeded):
   represents exactly.
 * KV-cache slots at or beyond a sequence's length hold NaN, so any read past the
   valid tokens poisons the output.
+* fp8 caches (``kv_dtype="fp8"``): the same fp32 draws divided by a per-tensor scale of
+  ``2^-6``, clamped to +-448 and rounded to OCP FP8 E4M3 codes (``torch.float8_e4m3fn``),
+  stored as uint8; unused slots hold the NaN code 0x7F.
 """
 
 from __future__ import annotations
@@ -81,7 +84,7 @@ def _lengths(rng: np.random.Generator, B: int, lo: int, hi: int) -> np.ndarray:
 
 
 def decode_contiguous_inputs(B: int, Hq: int, Hkv: int, D: int, cap: int, len_lo: int, len_hi: int,
-                             seed: int = 0, seqlens=None):
+                             seed: int = 0, seqlens=None, kv_dtype: str = "bf16"):
     """One query token per sequence and a dense cache ``[B,Hkv,cap,D]`` (bf16).
 
     Lengths are uniform in ``[len_lo, len_hi]`` unless ``seqlens`` is given; slots at
@@ -98,13 +101,32 @@ def decode_contiguous_inputs(B: int, Hq: int, Hkv: int, D: int, cap: int, len_lo
     for b in range(B):
         k[b, :, int(lens[b]):] = float("nan")
         v[b, :, int(lens[b]):] = float("nan")
-    return {"q": q, "k_cache": k, "v_cache": v, "seqlens": torch.from_numpy(lens),
-            "block_table": None, "block_size": cap, "max_seqlen": int(lens.max(initial=0))}
+    out = {"q": q, "k_cache": k, "v_cache": v, "seqlens": torch.from_numpy(lens),
+           "block_table": None, "block_size": cap, "max_seqlen": int(lens.max(initial=0))}
+    return _fp8_cache(out) if kv_dtype == "fp8" else out
+
+
+FP8_SCALE = 2.0 ** -6
+
+
+def _to_fp8(x: torch.Tensor) -> torch.Tensor:
+    """E4M3 codes (uint8) of ``x / FP8_SCALE`` (NaN stays NaN)."""
+    y = (x.float() / FP8_SCALE).clamp(-448.0, 448.0)
+    y = torch.where(torch.isnan(x.float()), x.float(), y)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def _fp8_cache(x: dict) -> dict:
+    x = dict(x)
+    x["k_cache"] = _to_fp8(x["k_cache"])
+    x["v_cache"] = _to_fp8(x["v_cache"])
+    x["k_scale"] = x["v_scale"] = FP8_SCALE
+    return x
 
 
 def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_lo: int, len_hi: int,
                         seed: int = 0, max_blocks: int | None = None, seqlens=None, extra_blocks: int = 0,
-                        device=None):
+                        device=None, kv_dtype: str = "bf16"):
     """One query token per sequence and a paged pool ``[num_blocks,Hkv,block_size,D]`` (bf16).
 
     The pool has ``sum(ceil(len/block_size)) + extra_blocks`` blocks; a seeded
@@ -114,6 +136,7 @@ def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_
 
     ``device`` (timing-only inputs): draw q and the pool with a generator on that device,
     seeded the same way, instead of on the CPU; lengths and the table are unchanged.
+    ``kv_dtype="fp8"`` returns the pool as E4M3 codes with ``k_scale``/``v_scale``.
     """
     rng = np.random.Generator(np.random.PCG64(seed))
     lens = _lengths(rng, B, len_lo, len_hi) if seqlens is None else np.asarray(seqlens, dtype=np.int32)
@@ -143,9 +166,10 @@ def decode_paged_inputs(B: int, Hq: int, Hkv: int, D: int, block_size: int, len_
         idx = torch.from_numpy(perm[used:].astype(np.int64)).to(k.device)
         k[idx] = float("nan")
         v[idx] = float("nan")
-    return {"q": q, "k_cache": k, "v_cache": v, "seqlens": torch.from_numpy(lens),
-            "block_table": torch.from_numpy(table), "block_size": block_size,
-            "max_seqlen": int(lens.max(initial=0)), "num_blocks": total}
+    out = {"q": q, "k_cache": k, "v_cache": v, "seqlens": torch.from_numpy(lens),
+           "block_table": torch.from_numpy(table), "block_size": block_size,
+           "max_seqlen": int(lens.max(initial=0)), "num_blocks": total}
+    return _fp8_cache(out) if kv_dtype == "fp8" else out
 
 
 def to_f64(t) -> np.ndarray:

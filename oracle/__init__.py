@@ -35,7 +35,7 @@ from .attention import (
     flash_blockwise_ref,
     allowed_mask,
 )
-from .kvcache import kv_cache_bytes_ref, paged_pool_blocks_ref
+from .kvcache import e4m3_decode, e4m3_value, kv_cache_bytes_ref, paged_pool_blocks_ref
 from .plan import decode_plan_ref, decode_heads_per_cta_ref, decode_schedule_ref
 
 __all__ = [
@@ -47,6 +47,8 @@ __all__ = [
     "allowed_mask",
     "kv_cache_bytes_ref",
     "paged_pool_blocks_ref",
+    "e4m3_value",
+    "e4m3_decode",
     "decode_plan_ref",
     "decode_schedule_ref",
     "decode_heads_per_cta_ref",

@@ -524,3 +524,37 @@ def test_decode_schedule_tiles_every_stream_once(case):
     if busy:
         # a segment's unit count is exact (t0 is unit-aligned, t1 aligned or the sequence end)
         assert max(busy) - min(busy) <= 1
+
+
+# ---------------------------------------------------------------- fp8 (E4M3) KV cache
+
+
+def test_e4m3_known_codes():
+    from oracle import e4m3_value
+
+    table = {0x00: 0.0, 0x80: -0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0,
+             0xB8: -1.0, 0x3C: 1.5, 0x40: 2.0, 0x7E: 448.0, 0xFE: -448.0, 0x77: 240.0, 0x30: 0.5}
+    for code, val in table.items():
+        assert e4m3_value(code) == val, hex(code)
+    assert math.isnan(e4m3_value(0x7F)) and math.isnan(e4m3_value(0xFF))
+
+
+def test_e4m3_decoder_matches_torch_float8():
+    # A library routine that implements the same format: every one of the 256 codes.
+    from oracle import e4m3_decode
+
+    codes = np.arange(256, dtype=np.uint8)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    mine = e4m3_decode(codes)
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(mine[ok], ref[ok])
+
+
+def test_e4m3_values_are_ordered_and_scaled():
+    from oracle import e4m3_decode
+
+    pos = e4m3_decode(np.arange(0x7F, dtype=np.uint8))  # 0 .. 448, NaN excluded
+    assert np.all(np.diff(pos) > 0)
+    assert np.array_equal(e4m3_decode(np.arange(0x80, 0xFF, dtype=np.uint8)), -pos)
+    assert np.array_equal(e4m3_decode(np.arange(0x7F, dtype=np.uint8), scale=0.25), pos * 0.25)
