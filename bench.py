@@ -409,6 +409,73 @@ def run_ours(args, rank, world, local):
             r["relative_to_mha"] = r["tokens_per_s"] / base
         assert device_status(clear=True) == 0
 
+    # Timing of the context measurements below: L2 flushed before each call, mean of `iters`.
+    def time_calls(fn, iters):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+        for _ in range(3):
+            flush_l2(1.0)
+            fn()
+        for i in range(iters):
+            flush_l2(float(i))
+            evs[i][0].record(stream)
+            fn()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(sum(a.elapsed_time(b) for a, b in evs) / iters, world)
+
+    # Sliding window (context, outside the timed region): the long-context prefill shape with a
+    # 4096-key window, and the paged decode workload attending to its last 2048 tokens.
+    win = None
+    if not args.no_window:
+        import numpy as np
+
+        WS, WW = 16384, 4096
+        wx = prefill_inputs(1, 64, 8, WS, WS, 128, dtype="bf16", seed=seed)
+        wq, wk, wv = wx["q"].to(dev), wx["k"].to(dev), wx["v"].to(dev)
+        wo = torch.empty_like(wq)
+        wl = torch.empty(wq.shape[:3], device=dev, dtype=torch.float32)
+        ms_p = time_calls(lambda: attn_fwd(wq, wk, wv, causal=True, o=wo, lse=wl, window=WW), args.sweep_iters)
+        pairs = float(np.minimum(np.arange(WS) + 1, WW).sum())
+        fl_w = 4.0 * 128 * 64 * pairs
+        del wx, wq, wk, wv, wo, wl
+        DW = 2048
+        ms_d = time_calls(lambda: attn_decode(paged["q"], paged["k_cache"], paged["v_cache"], paged["seqlens"],
+                                              max_seqlen=paged["max_seqlen"], block_table=paged["block_table"],
+                                              workspace=paged["ws"], o=paged["o"], lse=paged["lse"], window=DW),
+                          args.sweep_iters)
+        lens = paged["seqlens"].cpu().numpy().astype("int64")
+        dbytes = float(np.minimum(lens, DW).sum()) * S["Hkv"] * S["D"] * 4
+        win = {"prefill": {"workload": f"B=1 Hq=64 Hkv=8 S={WS} D=128 causal, window {WW}", "ms": ms_p,
+                           "TFLOP/s": fl_w / (ms_p * 1e-3) / 1e12,
+                           "frac": fl_w / (ms_p * 1e-3) / 1e12 / peaks["bf16_tflops"], "flops": fl_w},
+               "decode": {"workload": f"paged B=64 Hq=32 Hkv=8 D=128 block 16 len U[512,8192], window {DW}",
+                          "ms": ms_d, "GB/s": dbytes / (ms_d * 1e-3) / 1e9,
+                          "frac": dbytes / (ms_d * 1e-3) / 1e9 / peaks["hbm_gbs"], "kv_bytes": dbytes}}
+        torch.cuda.empty_cache()
+        assert device_status(clear=True) == 0
+
+    # FP8 (E4M3) KV cache (context, outside the timed region): the paged decode workload with
+    # its pool stored as E4M3 codes; bytes are the fp8 K/V of the valid tokens.
+    f8 = None
+    if not args.no_window:
+        from exact_attention_137_b200 import attn_decode_fp8
+
+        fx = decode_paged_inputs(S["B"], S["Hq"], S["Hkv"], S["D"], S["bs"], S["lo"], S["hi"], seed=seed,
+                                 device=dev, kv_dtype="fp8")
+        fg = {kk: (vv.to(dev) if isinstance(vv, torch.Tensor) else vv) for kk, vv in fx.items()}
+        ms_f = time_calls(lambda: attn_decode_fp8(fg["q"], fg["k_cache"], fg["v_cache"], fx["k_scale"], fx["v_scale"],
+                                                  fg["seqlens"], max_seqlen=fg["max_seqlen"],
+                                                  block_table=fg["block_table"], workspace=paged["ws"],
+                                                  o=paged["o"], lse=paged["lse"]), args.sweep_iters)
+        fbytes = float(fx["seqlens"].numpy().astype("int64").sum()) * S["Hkv"] * S["D"] * 2
+        f8 = {"workload": "paged B=64 Hq=32 Hkv=8 D=128 block 16 len U[512,8192], E4M3 K/V with per-tensor scales",
+              "ms": ms_f, "GB/s": fbytes / (ms_f * 1e-3) / 1e9, "frac": fbytes / (ms_f * 1e-3) / 1e9 / peaks["hbm_gbs"],
+              "kv_bytes": fbytes, "tokens_per_s": S["B"] / (ms_f * 1e-3),
+              "speedup_vs_bf16": per_call["decode_paged"] / ms_f}
+        del fx, fg
+        torch.cuda.empty_cache()
+        assert device_status(clear=True) == 0
+
     hbm = peaks["hbm_gbs"]
     tf_peak = peaks["bf16_tflops"]
     per_launch_ms = pre_ms / len(pre)
@@ -445,6 +512,8 @@ def run_ours(args, rank, world, local):
             "workload": "paged B=64 Hq=32 D=128 block 16 len U[512,8192], Hkv in {32 (MHA), 8 (GQA), 1 (MQA)}; "
                         "one decoded token per sequence; L2 flushed before each call",
             "rows": sweep},
+        "window": win,
+        "fp8_kv_decode": f8,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill sweep with q/k/v copied from pinned host memory and O/LSE copied back each step"},
         "gpu_launches": launches_per_step * args.steps,
@@ -465,6 +534,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode-sweep", action="store_true")
+    ap.add_argument("--no-window", action="store_true")
     ap.add_argument("--sweep-iters", type=int, default=30)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()

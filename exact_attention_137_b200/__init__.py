@@ -12,6 +12,7 @@ this package is a thin binding plus seeded synthetic inputs (``workloads``).
 from ._lib import (  # noqa: F401
     AttnError,
     attn_decode,
+    attn_decode_fp8,
     attn_fwd,
     decode_check,
     decode_plan,
@@ -27,6 +28,7 @@ from ._lib import (  # noqa: F401
 __all__ = [
     "AttnError",
     "attn_decode",
+    "attn_decode_fp8",
     "attn_fwd",
     "decode_check",
     "decode_plan",

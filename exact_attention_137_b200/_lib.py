@@ -49,6 +49,8 @@ _SIGS = {
                                  _c_int, _c_int, _vp]),
     "attn_decode_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                     _c_int, _c_float, _c_int, _vp, _size_t, _vp, _vp, _c_int, _vp]),
+    "attn_decode_fp8": (_c_int, [_vp, _vp, _vp, _c_float, _c_float, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _size_t, _vp, _vp, _vp]),
     "attn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                      _c_int, _c_float, _vp, _vp, _c_int, _vp]),
     "attn_decode_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int, _c_int, _c_int]),
@@ -254,6 +256,36 @@ def attn_decode(q, k_cache, v_cache, seqlens, max_seqlen: int, block_table=None,
                          workspace.numel() * workspace.element_size(), _ptr(o), _ptr(lse), _dtype_code(q),
                          ctypes.c_void_p(_stream_ptr(stream)))
     _check(st, "attn_decode")
+    return o, lse
+
+
+def attn_decode_fp8(q, k_cache, v_cache, k_scale: float, v_scale: float, seqlens, max_seqlen: int, block_table=None,
+                    block_size: int | None = None, scale: float | None = None, window: int = 0, workspace=None,
+                    o=None, lse=None, stream=None):
+    """Decode over an E4M3 KV cache (``k_cache``/``v_cache`` uint8 codes, layouts of
+    :func:`attn_decode`) with per-tensor scales.  Returns ``(o, lse)``."""
+    lib = load()
+    B, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    if k_cache.dtype != torch.uint8 or v_cache.dtype != torch.uint8 or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache/v_cache must be uint8 E4M3 codes of one shape")
+    if block_table is None:
+        bs, max_blocks, num_blocks = k_cache.shape[2], 1, B
+    else:
+        bs = k_cache.shape[2] if block_size is None else int(block_size)
+        max_blocks, num_blocks = block_table.shape[1], k_cache.shape[0]
+    if workspace is None:
+        workspace = decode_workspace(B, Hq, Hkv, D, max_seqlen, q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq), device=q.device, dtype=torch.float32)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib.attn_decode_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), float(k_scale), float(v_scale), _ptr(seqlens),
+                             _ptr(block_table), bs, max_blocks, num_blocks, int(max_seqlen), B, Hq, Hkv, D, sc,
+                             int(window), _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(o),
+                             _ptr(lse), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(st, "attn_decode_fp8")
     return o, lse
 
 

@@ -136,8 +136,8 @@ int launch_fwd_tc(const void* q, const void* k, const void* v, void* o, float* l
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = std::min(p.items, sms);  // persistent: one CTA per SM walks its share of the items
-  auto kern = attn::tc::fwd_tc_kernel<D>;
-  cudaError_t e = set_smem_once(kern, Lay::kAlloc, D == 64 ? 0 : 1);
+  auto kern = p.window > 0 ? attn::tc::fwd_tc_kernel<D, true> : attn::tc::fwd_tc_kernel<D, false>;
+  cudaError_t e = set_smem_once(kern, Lay::kAlloc, (D == 64 ? 0 : 1) + (p.window > 0 ? 2 : 0));
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   kern<<<grid, attn::tc::kThreads, Lay::kAlloc, st>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -199,12 +199,12 @@ WsLayout ws_layout(int B, int D, const DecodePlan& pl) {
   return w;
 }
 
-template <int D, int G>
+template <int D, int G, int KVB>
 int launch_decode(const attn::dec::Params& p, int ctas, cudaStream_t st) {
-  using Lay = attn::dec::Layout<D, G>;
-  auto kern = attn::dec::decode_kernel<D, G>;
-  const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3);
-  static bool done[64][8] = {};
+  using Lay = attn::dec::Layout<D, G, KVB>;
+  auto kern = attn::dec::decode_kernel<D, G, KVB>;
+  const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3) + (KVB == 1 ? 8 : 0);
+  static bool done[64][16] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -223,10 +223,20 @@ int launch_decode(const attn::dec::Params& p, int ctas, cudaStream_t st) {
 template <int D>
 int dispatch_decode_g(const attn::dec::Params& p, int G, int ctas, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode<D, 1>(p, ctas, st);
-    case 2: return launch_decode<D, 2>(p, ctas, st);
-    case 4: return launch_decode<D, 4>(p, ctas, st);
-    case 8: return launch_decode<D, 8>(p, ctas, st);
+    case 1: return launch_decode<D, 1, 2>(p, ctas, st);
+    case 2: return launch_decode<D, 2, 2>(p, ctas, st);
+    case 4: return launch_decode<D, 4, 2>(p, ctas, st);
+    case 8: return launch_decode<D, 8, 2>(p, ctas, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+// E4M3 caches: D = 128 and at most 4 query heads per CTA.
+int dispatch_decode_fp8(const attn::dec::Params& p, int G, int ctas, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode<128, 1, 1>(p, ctas, st);
+    case 2: return launch_decode<128, 2, 1>(p, ctas, st);
+    case 4: return launch_decode<128, 4, 1>(p, ctas, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
@@ -385,10 +395,16 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int D, int max_seqlen
   return ws_layout(B, D, pl).total;
 }
 
-int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
-                       const int* block_table, int block_size, int max_blocks, int num_blocks, int max_seqlen, int B,
-                       int Hq, int Hkv, int D, float scale, int window, void* workspace, size_t workspace_bytes,
-                       void* o, float* lse, int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// attn_decode_window and attn_decode_fp8.  kv_fp8: the cache holds E4M3 codes, dequantised
+// with k_scale and v_scale.
+int decode_impl(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
+                int block_size, int max_blocks, int num_blocks, int max_seqlen, int B, int Hq, int Hkv, int D,
+                float scale, int window, bool kv_fp8, float k_scale, float v_scale, void* workspace,
+                size_t workspace_bytes, void* o, float* lse, int dtype, void* stream) {
   if (window < 0) return ATTN_ERR_ARG;
   if (!q || !k_cache || !v_cache || !seqlens || !o) return ATTN_ERR_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || block_size <= 0 || max_seqlen < 0 || !std::isfinite(scale))
@@ -412,8 +428,8 @@ int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   attn::dec::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
-  p.kc = static_cast<const __nv_bfloat16*>(k_cache);
-  p.vc = static_cast<const __nv_bfloat16*>(v_cache);
+  p.kc = k_cache;
+  p.vc = v_cache;
   p.seqlens = seqlens;
   p.block_table = block_table;
   p.block_size = block_size;
@@ -425,7 +441,10 @@ int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, 
   p.Hkv = Hkv;
   p.nsub = (Hq / Hkv) / pl.G;
   p.window = window;
-  p.scale_log2 = scale * attn::kLog2e;
+  // E4M3 rows arrive in fp32 as value * 2^-120 (see e4m3_raw); both factors fold in here.
+  const float fac = kv_fp8 ? std::ldexp(1.0f, 120) : 1.0f;
+  p.scale_log2 = scale * attn::kLog2e * (kv_fp8 ? k_scale * fac : 1.0f);
+  p.v_fac = kv_fp8 ? v_scale * fac : 1.0f;
   const WsLayout wl = ws_layout(B, D, pl);
   const int sms = device_sms();
   if (sms <= 0) return ATTN_ERR_CUDA;
@@ -437,8 +456,35 @@ int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, 
   p.lse = lse;
   cudaStream_t st = as_stream(stream);
   const int ctas = plan_ctas(pl, sms);
+  if (kv_fp8) return dispatch_decode_fp8(p, pl.G, ctas, st);
   return D == 64 ? dispatch_decode_g<64>(p, pl.G, ctas, st) : dispatch_decode_g<128>(p, pl.G, ctas, st);
 }
+
+}  // namespace
+
+extern "C" {
+
+int attn_decode_window(const void* q, const void* k_cache, const void* v_cache, const int* seqlens,
+                       const int* block_table, int block_size, int max_blocks, int num_blocks, int max_seqlen, int B,
+                       int Hq, int Hkv, int D, float scale, int window, void* workspace, size_t workspace_bytes,
+                       void* o, float* lse, int dtype, void* stream) {
+  return decode_impl(q, k_cache, v_cache, seqlens, block_table, block_size, max_blocks, num_blocks, max_seqlen, B, Hq,
+                     Hkv, D, scale, window, false, 1.0f, 1.0f, workspace, workspace_bytes, o, lse, dtype, stream);
+}
+
+int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache, float k_scale, float v_scale,
+                    const int* seqlens, const int* block_table, int block_size, int max_blocks, int num_blocks,
+                    int max_seqlen, int B, int Hq, int Hkv, int D, float scale, int window, void* workspace,
+                    size_t workspace_bytes, void* o, float* lse, void* stream) {
+  if (!std::isfinite(k_scale) || !std::isfinite(v_scale) || !(k_scale > 0.f) || !(v_scale > 0.f))
+    return ATTN_ERR_ARG;
+  if (D != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hq > 0 && Hkv > 0 && Hq % Hkv == 0 && (Hq / Hkv) % 8 == 0) return ATTN_ERR_UNSUPPORTED;  // 8 heads per CTA
+  return decode_impl(q, k_cache, v_cache, seqlens, block_table, block_size, max_blocks, num_blocks, max_seqlen, B, Hq,
+                     Hkv, D, scale, window, true, k_scale, v_scale, workspace, workspace_bytes, o, lse, ATTN_BF16,
+                     stream);
+}
+
 
 int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int* seqlens, const int* block_table,
                 int block_size, int max_blocks, int num_blocks, int max_seqlen, int B, int Hq, int Hkv, int D,

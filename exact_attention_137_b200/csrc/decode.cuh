@@ -158,15 +158,16 @@ inline Walk walk_start_host(const LenOf& len_of, int B, int Y, long long total, 
 
 struct Params {
   const __nv_bfloat16* q;
-  const __nv_bfloat16* kc;
-  const __nv_bfloat16* vc;
+  const void* kc;  // bf16 values, or E4M3 codes (one byte each)
+  const void* vc;
   const int* seqlens;
   const int* block_table;  // nullptr: contiguous cache
   int block_size, max_blocks, num_blocks, max_seqlen;
   int B, Hq, Hkv;
   int nsub;  // query-head subgroups of G per KV head
   int window;  // > 0: attend to the last `window` cached tokens only
-  float scale_log2;
+  float scale_log2;  // scale * log2(e), times the K dequantisation factor for E4M3 caches
+  float v_fac;       // multiplies O: 1, or the V dequantisation factor for E4M3 caches
   float* ws_o;    // [grid][2][G][D] partial outputs per CTA slot
   float* ws_lse;  // [grid][2][G]
   unsigned int* ws_err;
@@ -183,12 +184,13 @@ struct SegSlots {
   int has[2];
 };
 
-template <int D, int G>
+template <int D, int G, int KVB>
 struct Layout {
-  static constexpr int kRow = D * 2;
+  static constexpr int kRow = D * KVB;                     // bytes of one cached K (or V) row
   static constexpr int kStageBytes = kStageTokens * kRow;  // K (or V) bytes of one stage
   static constexpr int kSlotBytes = 2 * kStageBytes;       // a stage: K rows, then V rows
-  static constexpr int kQBytes = G * kRow;                 // the segment's query rows
+  static constexpr int kQRow = D * 2;                      // a bf16 query row
+  static constexpr int kQBytes = G * kQRow;                // the segment's query rows
   static constexpr int kQ = kStages * kSlotBytes;
   static constexpr int kBar = kQ + kStages * kQBytes;
   static constexpr int kMisc = kBar + 2 * kStages * 8;
@@ -221,6 +223,16 @@ __device__ __forceinline__ int checked_len(const Params& p, int b, bool report) 
 __device__ __forceinline__ int span_len(const Params& p, int b, bool report) {
   const int len = checked_len(p, b, report);
   return (p.window > 0 && len > p.window) ? p.window : len;
+}
+
+// E4M3 code `k` of the word w as an fp32 whose value is the code's value times 2^-120: the
+// sign moves to bit 31 and the 7 exponent-and-mantissa bits to bits 26..20, so the fp32
+// exponent field is the E4M3 one (bias 127 instead of 7), and E4M3 subnormals land on fp32
+// subnormals with the same factor.  The factor is folded into the score scale and into O.
+// The NaN code S.1111.111 becomes the finite 480 * 2^-120.
+__device__ __forceinline__ float e4m3_raw(uint32_t w, int k) {
+  const int t = (int)__byte_perm(w, 0u, ((uint32_t)k << 12) | 0x444u);  // code in bits 31..24
+  return __int_as_float((t >> 4) & (int)0x87F00000);
 }
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -317,11 +329,13 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory");
 }
 
-template <int D, int G>
+template <int D, int G, int KVB>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   // Lanes per token row: 8, except D=128 with 8 heads per CTA, where 16 lanes halve the
-  // per-lane query and accumulator registers.
+  // per-lane query and accumulator registers.  KVB: bytes per cached element (2: bf16,
+  // 1: E4M3, whose 16-byte slice holds 16 elements, so lane j owns elements 16j..16j+15).
   constexpr int LPT = (D == 128 && G == 8) ? 16 : 8;
+  static_assert(KVB == 2 || (KVB == 1 && D == 128 && LPT == 8), "E4M3 caches: D = 128, at most 4 heads per CTA");
   constexpr int EPL = D / LPT;     // elements of a row per lane (16 at D=128, 8 at D=64)
   constexpr int WPL = EPL / 2;     // 32-bit words (bf16 pairs) per lane per row
   constexpr int TOK = LPT / G;     // tokens per lane group per step
@@ -331,7 +345,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   constexpr int kCon = kConsumerWarps * 32;
   static_assert(G <= LPT && TOK * G == LPT, "heads per CTA must divide the lanes per token");
   static_assert(EPL % 8 == 0, "each lane reads whole 16-byte slices");
-  using L = Layout<D, G>;
+  using L = Layout<D, G, KVB>;
+  // One cached row's elements of this lane as fp32 pairs (for E4M3: times 2^-120).
+  auto load_row = [&](uint32_t row, int jl, uint64_t(&out)[EPL / 2]) {
+    if constexpr (KVB == 2) {
+#pragma unroll
+      for (int v4 = 0; v4 < EPL / 8; ++v4) {
+        const uint4 w = lds128(row + 16u * (jl + LPT * v4));
+        out[4 * v4 + 0] = f2pack(bf16lo(w.x), bf16hi(w.x));
+        out[4 * v4 + 1] = f2pack(bf16lo(w.y), bf16hi(w.y));
+        out[4 * v4 + 2] = f2pack(bf16lo(w.z), bf16hi(w.z));
+        out[4 * v4 + 3] = f2pack(bf16lo(w.w), bf16hi(w.w));
+      }
+    } else {
+      const uint4 w = lds128(row + 16u * jl);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        out[2 * q] = f2pack(e4m3_raw(ws[q], 0), e4m3_raw(ws[q], 1));
+        out[2 * q + 1] = f2pack(e4m3_raw(ws[q], 2), e4m3_raw(ws[q], 3));
+      }
+    }
+  };
+  // Which element of the row the lane's e-th value is.
+  auto elem_of = [&](int jl, int e) -> int {
+    return KVB == 2 ? 8 * (jl + LPT * (e >> 3)) + (e & 7) : EPL * jl + e;
+  };
 
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
@@ -428,8 +467,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
               const uint32_t bytes = (uint32_t)run * L::kRow;
               const uint32_t dst = (uint32_t)(tok - a) * L::kRow;
               mbar_expect_tx(full_bar(s), 2u * bytes);
-              bulk_load(dk + dst, p.kc + off, bytes, full_bar(s));
-              bulk_load(dv + dst, p.vc + off, bytes, full_bar(s));
+              bulk_load(dk + dst, static_cast<const uint8_t*>(p.kc) + off * KVB, bytes, full_bar(s));
+              bulk_load(dv + dst, static_cast<const uint8_t*>(p.vc) + off * KVB, bytes, full_bar(s));
             }
           }
           tok += run;
@@ -494,7 +533,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
         for (int hh = 0; hh < G; ++hh)
 #pragma unroll
           for (int v4 = 0; v4 < EPL / 8; ++v4) {
-            const uint4 wq = lds128(sq + hh * L::kRow + 16u * (j + LPT * v4));
+            // the bf16 query elements this lane owns, in the order of its K elements
+            const uint32_t off = KVB == 2 ? 16u * (j + LPT * v4) : 2u * EPL * j + 16u * v4;
+            const uint4 wq = lds128(sq + hh * L::kQRow + off);
             q2[hh][4 * v4 + 0] = f2pack(bf16lo(wq.x), bf16hi(wq.x));
             q2[hh][4 * v4 + 1] = f2pack(bf16lo(wq.y), bf16hi(wq.y));
             q2[hh][4 * v4 + 2] = f2pack(bf16lo(wq.z), bf16hi(wq.z));
@@ -518,14 +559,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             uint64_t k2[WPL];
-#pragma unroll
-            for (int v4 = 0; v4 < EPL / 8; ++v4) {
-              const uint4 wk = lds128(sk + (uint32_t)((x ? tb1 : tb0) + tt) * L::kRow + 16u * (j + LPT * v4));
-              k2[4 * v4 + 0] = f2pack(bf16lo(wk.x), bf16hi(wk.x));
-              k2[4 * v4 + 1] = f2pack(bf16lo(wk.y), bf16hi(wk.y));
-              k2[4 * v4 + 2] = f2pack(bf16lo(wk.z), bf16hi(wk.z));
-              k2[4 * v4 + 3] = f2pack(bf16lo(wk.w), bf16hi(wk.w));
-            }
+            load_row(sk + (uint32_t)((x ? tb1 : tb0) + tt) * L::kRow, j, k2);
 #pragma unroll
             for (int hh = 0; hh < G; ++hh) {
               uint64_t d2 = fmul2(q2[hh][0], k2[0]);
@@ -566,14 +600,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
           for (int x = 0; x < 2; ++x) {
             uint64_t v2[WPL];
             const int tok = (x ? tb1 : tb0) + tt;
-#pragma unroll
-            for (int v4 = 0; v4 < EPL / 8; ++v4) {
-              const uint4 wv = lds128(sv + (uint32_t)tok * L::kRow + 16u * (j + LPT * v4));
-              v2[4 * v4 + 0] = f2pack(bf16lo(wv.x), bf16hi(wv.x));
-              v2[4 * v4 + 1] = f2pack(bf16lo(wv.y), bf16hi(wv.y));
-              v2[4 * v4 + 2] = f2pack(bf16lo(wv.z), bf16hi(wv.z));
-              v2[4 * v4 + 3] = f2pack(bf16lo(wv.w), bf16hi(wv.w));
-            }
+            load_row(sv + (uint32_t)tok * L::kRow, j, v2);
             const bool tv = (x == 0 || has1) && tok < nv;
 #pragma unroll
             for (int hh = 0; hh < G; ++hh) {
@@ -629,7 +656,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
         for (int hh = 0; hh < G; ++hh)
 #pragma unroll
           for (int e = 0; e < EPL; ++e)
-            a_s[(warp * G + hh) * D + 8 * (j + LPT * (e >> 3)) + (e & 7)] = accf[hh][e];
+            a_s[(warp * G + hh) * D + elem_of(j, e)] = accf[hh][e];
       }
     }
     consumer_sync<kCon>();
@@ -650,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
           O += a_s[(w4 * G + hh) * D + d] * sc;
         }
       }
-      const float o_val = Lsum > 0.f ? O / Lsum : 0.f;
+      const float o_val = Lsum > 0.f ? (KVB == 2 ? O / Lsum : O / Lsum * p.v_fac) : 0.f;
       const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
       if (sg.slot < 0) {  // the whole stream: write the result directly
         p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);

@@ -146,9 +146,11 @@ __device__ __forceinline__ int kv_tiles(const Params& p, int t) {
 }
 
 // First KV tile any row of query tile t can see: 0, or with a sliding window the tile of the
-// first row's earliest key p - W + 1 (p = row + Sk - Sq).
+// first row's earliest key p - W + 1 (p = row + Sk - Sq).  kWindow selects the kernel built
+// for windowed calls; the plain kernel carries none of the window arithmetic.
+template <bool kWindow>
 __device__ __forceinline__ int kv_first(const Params& p, int t) {
-  if (p.window <= 0) return 0;
+  if (!kWindow || p.window <= 0) return 0;
   const long long first = (long long)t * BM + (long long)p.Sk - p.Sq - p.window + 1;
   return first <= 0 ? 0 : (int)(first / BN);
 }
@@ -156,6 +158,7 @@ __device__ __forceinline__ int kv_first(const Params& p, int t) {
 // Work items, longest first under a causal mask.  Items [0, items_a): two heads of one KV
 // group, same query tile.  Items [items_a, ...): the leftover head of an odd group, query
 // tiles 2t and 2t+1.
+template <bool kWindow>
 __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
   Item it;
   const int g = p.g;
@@ -183,7 +186,7 @@ __device__ __forceinline__ Item decode_item(const Params& p, int idx) {
   }
   for (int i = 0; i < 2; ++i) {
     const int hi = it.t[i] < p.nq ? kv_tiles(p, it.t[i]) : 0;
-    it.f[i] = it.t[i] < p.nq ? kv_first(p, it.t[i]) : 0;
+    it.f[i] = it.t[i] < p.nq ? kv_first<kWindow>(p, it.t[i]) : 0;
     if (it.f[i] > hi) it.f[i] = hi;
     it.n[i] = hi - it.f[i];
   }
@@ -197,8 +200,15 @@ struct Span {
   int F, N, st[2];
 };
 
+template <bool kWindow>
 __device__ __forceinline__ Span item_span(const Item& it) {
   Span sp;
+  if (!kWindow) {  // every slot starts at tile 0
+    sp.F = 0;
+    sp.N = max(it.n[0], it.n[1]);
+    sp.st[0] = sp.st[1] = 0;
+    return sp;
+  }
   int lo = 0x7fffffff, hi = 0;
   for (int i = 0; i < 2; ++i)
     if (it.n[i] > 0) {
@@ -248,7 +258,7 @@ __device__ __forceinline__ void exp_chunk(const uint32_t (&v)[32], uint32_t* out
   }
 }
 
-template <int D>
+template <int D, bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -320,8 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; alive; ++r) {
           const int idx = item_of(r);
           if (idx >= p.items) break;
-          const Item it = decode_item(p, idx);
-          const Span sp = item_span(it);
+          const Item it = decode_item<kWindow>(p, idx);
+          const Span sp = item_span<kWindow>(it);
           const int N = sp.N;
           if (N == 0) continue;
           // Q_i of this item replaces the previous one once slot i's S MMAs are done with it.
@@ -425,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (;; ++rr) {
             const int idx = item_of(rr);
             if (idx >= p.items) return false;
-            out = decode_item(p, idx);
+            out = decode_item<kWindow>(p, idx);
             if (out.n[0] > 0 || out.n[1] > 0) return true;
           }
         };
@@ -434,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool have = next_item(r, it);
         bool started = false;  // S_i(0) of the current item was issued by the previous item's last step
         while (ok && have) {
-          const Span sp = item_span(it);
+          const Span sp = item_span<kWindow>(it);
           const int N = sp.N;
           int r2 = r + 1;
           Item nx;
@@ -445,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // epilogue executes.  Otherwise the next item starts with both S MMAs together.
           bool chain = false;
           if (have_next && it.n[0] > 0 && it.n[1] > 0 && nx.n[0] > 0 && nx.n[1] > 0) {
-            const Span spn = item_span(nx);
+            const Span spn = item_span<kWindow>(nx);
             chain = sp.st[0] + it.n[0] == N && sp.st[1] + it.n[1] == N && spn.st[0] == 0 && spn.st[1] == 0;
           }
           const int pnext = pos + 2 * N;  // ring position of the next item's K_0
@@ -537,9 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int r = 0; ok; ++r) {
       const int idx = item_of(r);
       if (idx >= p.items) break;
-      const Item it = decode_item(p, idx);
+      const Item it = decode_item<kWindow>(p, idx);
       const int n = i ? it.n[1] : it.n[0];
-      const int f = i ? it.f[1] : it.f[0];  // first KV tile
+      const int f = kWindow ? (i ? it.f[1] : it.f[0]) : 0;  // first KV tile
       const int t = i ? it.t[1] : it.t[0];
       const int h = i ? it.h[1] : it.h[0];
       if (t >= p.nq) continue;  // this slot has no query tile in the item
@@ -547,8 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long long key_limit = p.causal ? (long long)qrow + p.Sk - p.Sq : (long long)p.Sk - 1;
       const long long tile_limit = p.causal ? (long long)t * BM + p.Sk - p.Sq : (long long)p.Sk - 1;
       // Sliding window: this row's first visible key, and the largest first key of the tile's rows.
-      const long long key_first = p.window > 0 ? (long long)qrow + p.Sk - p.Sq - p.window + 1 : 0;
-      const long long tile_first = p.window > 0 ? (long long)t * BM + BM - 1 + p.Sk - p.Sq - p.window + 1 : 0;
+      const long long key_first = kWindow ? (long long)qrow + p.Sk - p.Sq - p.window + 1 : 0;
+      const long long tile_first = kWindow ? (long long)t * BM + BM - 1 + p.Sk - p.Sq - p.window + 1 : 0;
       const float c = p.scale_log2;
       const uint64_t c2 = f2pack(c, c);
       // l: fp32 row sum (for the LSE); lr: row sum of the bf16 P that the tensor core
@@ -560,15 +570,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int kv0 = (f + j) * BN;
         // Mask only tiles that reach past the last key or the causal diagonal, or (window) start
         // before some row's first key.
-        const bool masked = (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk || (long long)kv0 < tile_first;
+        const bool masked =
+            (long long)kv0 + BN - 1 > tile_limit || kv0 + BN > p.Sk || (kWindow && (long long)kv0 < tile_first);
         // Keys lo..hi of a 32-key chunk are visible to this row: compares against constants.
         auto mask_chunk = [&](uint32_t(&v)[32], int q4) {
           const long long lim = (key_limit < (long long)p.Sk - 1 ? key_limit : (long long)p.Sk - 1) - kv0 - q4 * 32;
           const int cl = (int)(lim < -1 ? -1 : (lim > 32 ? 32 : lim));
-          const long long flo = key_first - kv0 - q4 * 32;
-          const int cf = (int)(flo < 0 ? 0 : (flo > 33 ? 33 : flo));
+          if (kWindow) {
+            const long long flo = key_first - kv0 - q4 * 32;
+            const int cf = (int)(flo < 0 ? 0 : (flo > 33 ? 33 : flo));
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = (e > cl || e < cf) ? __float_as_uint(-INFINITY) : v[e];
+            for (int e = 0; e < 32; ++e) v[e] = (e > cl || e < cf) ? __float_as_uint(-INFINITY) : v[e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) v[e] = e > cl ? __float_as_uint(-INFINITY) : v[e];
+          }
         };
         auto publish = [&](const uint32_t(&w)[32], uint32_t col, uint32_t b) {
           tmem_st32(tS + col, w);

@@ -146,6 +146,25 @@ int attn_decode_window(const void* q, const void* k_cache, const void* v_cache,
                        void* workspace, size_t workspace_bytes,
                        void* o, float* lse, int dtype, void* stream);
 
+/* attn_decode_fp8: attn_decode_window over an fp8 KV cache (CSDN «注意力变体深挖», 追问4,
+ * lists quantising the KV cache to fp8 among the long-context optimisations; the format
+ * is this library's reading).  k_cache and v_cache hold one OCP FP8 E4M3 code per element
+ * (1 byte; sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, no
+ * infinities), in the layouts of attn_decode; the cached value is code * k_scale
+ * (resp. v_scale), one positive fp32 scale per tensor.  q, o and lse are as in
+ * attn_decode (bf16 q and o).  The NaN code S.1111.111 is read as the finite value 480
+ * (it never propagates).  D must be 128 and Hq/Hkv must not be a multiple of 8
+ * (ATTN_ERR_UNSUPPORTED otherwise).  Scores and sums are fp32, as in attn_decode.
+ * Returns the codes of attn_decode_window, plus ATTN_ERR_ARG for a scale that is not a
+ * positive finite number. */
+int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
+                    float k_scale, float v_scale,
+                    const int* seqlens, const int* block_table,
+                    int block_size, int max_blocks, int num_blocks, int max_seqlen,
+                    int B, int Hq, int Hkv, int D, float scale, int window,
+                    void* workspace, size_t workspace_bytes,
+                    void* o, float* lse, void* stream);
+
 /* attn_decode_noalloc: the same decode as attn_decode, for callers that cannot allocate
  * device memory at all -- for example code running inside an allocator callback, a
  * real-time loop that must not risk the implicit synchronisation a cudaMalloc can cause,

@@ -195,3 +195,74 @@ def test_window_longer_than_every_sequence_is_plain_decode(cuda_lib):
                          block_table=g["block_table"], block_size=g["block_size"], window=900)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------- fp8 (E4M3) KV cache
+
+
+def _fp8_ref(x, window=0):
+    from oracle import e4m3_decode
+
+    bt = None if x["block_table"] is None else x["block_table"].numpy()
+    kc = e4m3_decode(x["k_cache"].numpy(), x["k_scale"])
+    vc = e4m3_decode(x["v_cache"].numpy(), x["v_scale"])
+    return decode_ref(to_f64(x["q"]), kc, vc, x["seqlens"].numpy(), block_table=bt, block_size=x["block_size"],
+                      window=window)
+
+
+@pytest.mark.parametrize("case", [
+    # kind, B, Hq, Hkv, lengths, window, block size
+    ("contiguous", 3, 32, 8, [1000, 1, 257], 0, None),
+    ("paged", 4, 32, 8, [512, 8192, 77, 3000], 0, 16),
+    ("paged", 2, 16, 8, [23, 101], 0, 5),             # two heads per CTA, odd pages
+    ("paged", 2, 8, 8, [640, 129], 0, 16),            # MHA
+    ("paged", 3, 32, 8, [4000, 700, 33], 1000, 16),   # with a window
+])
+def test_fp8(cuda_lib, case):
+    from exact_attention_137_b200 import attn_decode_fp8
+
+    kind, B, Hq, Hkv, lens, W, bs = case
+    if kind == "contiguous":
+        x = decode_contiguous_inputs(B, Hq, Hkv, 128, max(lens), 0, 0, seed=7, seqlens=lens, kv_dtype="fp8")
+    else:
+        x = decode_paged_inputs(B, Hq, Hkv, 128, bs, 0, max(lens), seed=7, seqlens=lens, extra_blocks=2,
+                                kv_dtype="fp8")
+    g = _gpu(x)
+    o, lse = attn_decode_fp8(g["q"], g["k_cache"], g["v_cache"], x["k_scale"], x["v_scale"], g["seqlens"],
+                             max_seqlen=g["max_seqlen"], block_table=g["block_table"], block_size=g["block_size"],
+                             window=W)
+    torch.cuda.synchronize()
+    compare(o, lse, *_fp8_ref(x, W), BF16_TOL, f"fp8 {case[:2]}")
+    assert device_status(clear=True) == 0
+
+
+def test_fp8_every_code_and_subnormals(cuda_lib):
+    # One sequence whose K and V rows run through all 254 finite codes, scale 2^-3.
+    from exact_attention_137_b200 import attn_decode_fp8
+
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    n = 254
+    kc = np.resize(codes, (1, 1, n, 128))
+    vc = np.resize(np.roll(codes, 37), (1, 1, n, 128))
+    x = {"q": torch.randn(1, 4, 128, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16),
+         "k_cache": torch.from_numpy(kc.copy()), "v_cache": torch.from_numpy(vc.copy()),
+         "seqlens": torch.tensor([n], dtype=torch.int32), "block_table": None, "block_size": n,
+         "k_scale": 0.125 / 64, "v_scale": 2.0 ** -7}
+    g = _gpu(x)
+    o, lse = attn_decode_fp8(g["q"], g["k_cache"], g["v_cache"], x["k_scale"], x["v_scale"], g["seqlens"],
+                             max_seqlen=n)
+    torch.cuda.synchronize()
+    compare(o, lse, *_fp8_ref(x), BF16_TOL, "fp8 all codes")
+
+
+def test_fp8_rejects_unsupported(cuda_lib):
+    from exact_attention_137_b200 import attn_decode_fp8
+
+    x = decode_paged_inputs(1, 32, 1, 128, 16, 0, 40, seed=1, seqlens=[40], kv_dtype="fp8")  # MQA: 8 heads per CTA
+    g = _gpu(x)
+    with pytest.raises(_lib.AttnError):
+        attn_decode_fp8(g["q"], g["k_cache"], g["v_cache"], 1.0, 1.0, g["seqlens"], max_seqlen=40,
+                        block_table=g["block_table"])
+    with pytest.raises(_lib.AttnError):
+        attn_decode_fp8(g["q"], g["k_cache"], g["v_cache"], 0.0, 1.0, g["seqlens"], max_seqlen=40,
+                        block_table=g["block_table"])
