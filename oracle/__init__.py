@@ -35,11 +35,13 @@ from .attention import (
     flash_blockwise_ref,
     allowed_mask,
 )
+from .backward import attention_bwd_ref
 from .kvcache import e4m3_decode, e4m3_value, kv_cache_bytes_ref, paged_pool_blocks_ref
 from .plan import decode_plan_ref, decode_heads_per_cta_ref, decode_schedule_ref
 
 __all__ = [
     "attention_ref",
+    "attention_bwd_ref",
     "attention_rows_ref",
     "brute_force_attention",
     "decode_ref",

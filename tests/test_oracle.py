@@ -558,3 +558,77 @@ def test_e4m3_values_are_ordered_and_scaled():
     assert np.all(np.diff(pos) > 0)
     assert np.array_equal(e4m3_decode(np.arange(0x80, 0xFF, dtype=np.uint8)), -pos)
     assert np.array_equal(e4m3_decode(np.arange(0x7F, dtype=np.uint8), scale=0.25), pos * 0.25)
+
+
+# ---------------------------------------------------------------- backward (recomputation)
+
+
+def _loss_and_grads(q, k, v, dout, **kw):
+    from oracle import attention_bwd_ref
+
+    o, _ = attention_ref(q, k, v, **kw)
+    return float(np.sum(o * dout)), attention_bwd_ref(q, k, v, dout, **kw)
+
+
+@pytest.mark.parametrize("kw", [dict(causal=False), dict(causal=True), dict(causal=True, window=2),
+                                dict(causal=True, scale=0.9)])
+def test_backward_matches_finite_differences(kw):
+    # L = sum(dO * O): its gradient w.r.t. Q, K, V is what the backward returns.
+    q, k, v, do = _rand((1, 4, 5, 3), 110), _rand((1, 2, 7, 3), 111), _rand((1, 2, 7, 3), 112), _rand((1, 4, 5, 3), 113)
+    _, (dq, dk, dv) = _loss_and_grads(q, k, v, do, **kw)
+    eps = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args = dict(q=q, k=k, v=v)
+            args[name] = xp
+            lp, _ = _loss_and_grads(args["q"], args["k"], args["v"], do, **kw)
+            args[name] = xm
+            lm, _ = _loss_and_grads(args["q"], args["k"], args["v"], do, **kw)
+            assert abs((lp - lm) / (2 * eps) - g[idx]) < 1e-7, (name, idx)
+
+
+def test_backward_matches_torch_autograd():
+    # A library routine: torch autograd through an explicit fp64 masked softmax.
+    from oracle import attention_bwd_ref
+
+    q, k, v, do = _rand((2, 6, 9, 8), 114), _rand((2, 2, 11, 8), 115), _rand((2, 2, 11, 8), 116), _rand((2, 6, 9, 8), 117)
+    qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kr, vr = kt.repeat_interleave(3, dim=1), vt.repeat_interleave(3, dim=1)
+    s = qt @ kr.transpose(-1, -2) / math.sqrt(8)
+    mask = torch.ones(9, 11, dtype=torch.bool).tril(diagonal=2)
+    o = torch.softmax(s.masked_fill(~mask, float("-inf")), dim=-1) @ vr
+    o.backward(torch.tensor(do))
+    dq, dk, dv = attention_bwd_ref(q, k, v, do, causal=True)
+    for mine, ref in ((dq, qt.grad), (dk, kt.grad), (dv, vt.grad)):
+        assert np.max(np.abs(mine - ref.numpy())) < 1e-12
+
+
+def test_backward_identities():
+    # Softmax rows sum to one, so sum_j dV_j = sum_i dO_i (rows with keys) and sum_j dK_j = 0;
+    # adding one vector to every key leaves dQ unchanged.
+    from oracle import attention_bwd_ref
+
+    q, k, v, do = _rand((1, 4, 12, 6), 118), _rand((1, 2, 12, 6), 119), _rand((1, 2, 12, 6), 120), _rand((1, 4, 12, 6), 121)
+    dq, dk, dv = attention_bwd_ref(q, k, v, do, causal=True)
+    for kh in range(2):
+        assert np.max(np.abs(dk[0, kh].sum(axis=0))) < 1e-12
+        assert np.max(np.abs(dv[0, kh].sum(axis=0) - do[0, 2 * kh:2 * kh + 2].sum(axis=(0, 1)))) < 1e-12
+    dq2, _, _ = attention_bwd_ref(q, k + _rand((6,), 122), v, do, causal=True)
+    assert np.max(np.abs(dq2 - dq)) < 1e-12
+
+
+def test_planted_backward_dropped_delta_is_caught(monkeypatch):
+    import oracle.backward as ob
+
+    real_sum = np.sum
+    fake = types.SimpleNamespace(**{n: getattr(np, n) for n in dir(np) if not n.startswith("__")})
+    fake.sum = lambda a, axis=None: real_sum(a, axis=axis) * 0.0  # Delta = 0
+    monkeypatch.setattr(ob, "np", fake)
+    q, k, v, do = _rand((1, 2, 4, 3), 123), _rand((1, 2, 4, 3), 124), _rand((1, 2, 4, 3), 125), _rand((1, 2, 4, 3), 126)
+    dq, _, _ = ob.attention_bwd_ref(q, k, v, do)
+    monkeypatch.undo()
+    dq_ok, _, _ = ob.attention_bwd_ref(q, k, v, do)
+    assert np.max(np.abs(dq - dq_ok)) > 1e-3
