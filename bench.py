@@ -454,6 +454,26 @@ def run_ours(args, rank, world, local):
         torch.cuda.empty_cache()
         assert device_status(clear=True) == 0
 
+    # Backward with recomputation (context, outside the timed region): the GQA variant of the
+    # prefill sweep; algorithmic FLOPs = 2.5x the forward's (five products of the visible pairs).
+    bwd = None
+    if not args.no_window:
+        from exact_attention_137_b200 import attn_bwd
+
+        c = pre[1] if len(pre) > 1 else pre[0]
+        attn_fwd(c["q"], c["k"], c["v"], causal=True, o=c["o"], lse=c["lse"])
+        gdo = torch.randn(c["q"].shape, device=dev, generator=torch.Generator(device=dev).manual_seed(seed + 7)).to(
+            torch.bfloat16)
+        gq, gk, gv = torch.empty_like(c["q"]), torch.empty_like(c["k"]), torch.empty_like(c["v"])
+        ms_b = time_calls(lambda: attn_bwd(c["q"], c["k"], c["v"], c["o"], c["lse"], gdo, causal=True, dq=gq, dk=gk,
+                                           dv=gv), args.sweep_iters)
+        fl_b = 2.5 * fl_call
+        bwd = {"workload": f"B=2 Hq=32 Hkv={c['hkv']} S=2048 D=128 causal, dQ dK dV from O, LSE, dO", "ms": ms_b,
+               "TFLOP/s": fl_b / (ms_b * 1e-3) / 1e12, "frac": fl_b / (ms_b * 1e-3) / 1e12 / peaks["bf16_tflops"],
+               "flops": fl_b, "tensor_path": "mma.sync m16n8k16 bf16 (warp-level)"}
+        del gdo, gq, gk, gv
+        assert device_status(clear=True) == 0
+
     # FP8 (E4M3) KV cache (context, outside the timed region): the paged decode workload with
     # its pool stored as E4M3 codes; bytes are the fp8 K/V of the valid tokens.
     f8 = None
@@ -514,6 +534,7 @@ def run_ours(args, rank, world, local):
             "rows": sweep},
         "window": win,
         "fp8_kv_decode": f8,
+        "backward": bwd,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill sweep with q/k/v copied from pinned host memory and O/LSE copied back each step"},
         "gpu_launches": launches_per_step * args.steps,

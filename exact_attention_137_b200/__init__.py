@@ -11,6 +11,7 @@ this package is a thin binding plus seeded synthetic inputs (``workloads``).
 
 from ._lib import (  # noqa: F401
     AttnError,
+    attn_bwd,
     attn_decode,
     attn_decode_fp8,
     attn_fwd,
@@ -27,6 +28,7 @@ from ._lib import (  # noqa: F401
 
 __all__ = [
     "AttnError",
+    "attn_bwd",
     "attn_decode",
     "attn_decode_fp8",
     "attn_fwd",

@@ -49,6 +49,9 @@ _SIGS = {
                                  _c_int, _c_int, _vp]),
     "attn_decode_window": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
                                     _c_int, _c_float, _c_int, _vp, _size_t, _vp, _vp, _c_int, _vp]),
+    "attn_bwd_workspace_bytes": (_size_t, [_c_int, _c_int, _c_int]),
+    "attn_bwd": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
+                          _c_float, _c_int, _c_int, _vp, _size_t, _vp]),
     "attn_decode_fp8": (_c_int, [_vp, _vp, _vp, _c_float, _c_float, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_float, _c_int, _vp, _size_t, _vp, _vp, _vp]),
     "attn_decode_noalloc": (_c_int, [_vp, _vp, _vp, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -165,6 +168,31 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
                       1 if causal else 0, _dtype_code(q), ctypes.c_void_p(_stream_ptr(stream)))
     _check(st, "attn_fwd")
     return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None, window: int = 0,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients ``(dq, dk, dv)`` of :func:`attn_fwd` given its ``o``, ``lse`` and ``dout``."""
+    lib = load()
+    B, Hq, Sq, D = q.shape
+    _, Hkv, Sk, _ = k.shape
+    for t in (q, k, v, o, dout, lse):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("inputs must be contiguous CUDA tensors")
+    if q.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise TypeError("bf16 q/k/v/o/dout and fp32 lse")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(1, int(lib.attn_bwd_workspace_bytes(B, Hq, Sq))), dtype=torch.uint8,
+                                device=q.device)
+    sc = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq,
+                      Hkv, Sq, Sk, D, sc, 1 if causal else 0, int(window), _ptr(workspace),
+                      workspace.numel() * workspace.element_size(), ctypes.c_void_p(_stream_ptr(stream)))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
 
 
 # ------------------------------------------------------------------ decode

@@ -14,6 +14,7 @@
 
 #include "../../include/attn.h"
 #include "common.cuh"
+#include "bwd.cuh"
 #include "decode.cuh"
 #include "prefill_simt.cuh"
 #include "prefill_tc.cuh"
@@ -151,6 +152,27 @@ int launch_fwd_simt(const void* q, const void* k, const void* v, void* o, float*
   attn::simt::fwd_simt_kernel<T, D><<<grid, attn::simt::kRowsPerBlock * 32, 0, st>>>(
       static_cast<const T*>(q), static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(o), lse,
       Hq, Hkv, Sq, Sk, scale * attn::kLog2e, causal ? 1 : 0, causal ? window : 0);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+
+template <int D>
+int launch_bwd(const attn::bwd::Params& p, cudaStream_t st) {
+  constexpr int kTileBytes = attn::bwd::kRows * D * 2;
+  const long long rows = (long long)p.B * p.Hq * p.Sq;
+  attn::bwd::delta_kernel<D><<<(unsigned)cdiv(rows, 8), 256, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  auto kdkdv = attn::bwd::dkdv_kernel<D>;
+  auto kdq = attn::bwd::dq_kernel<D>;
+  const int smem_kv = 4 * kTileBytes + 2 * attn::bwd::kRows * (int)sizeof(float);
+  const int smem_q = 4 * kTileBytes;
+  if (set_smem_once(kdkdv, smem_kv, D == 64 ? 4 : 5) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (set_smem_once(kdq, smem_q, D == 64 ? 6 : 7) != cudaSuccess) return ATTN_ERR_CUDA;
+  dim3 gkv((unsigned)cdiv(p.Sk, attn::bwd::kRows), (unsigned)(p.B * p.Hkv));
+  kdkdv<<<gkv, attn::bwd::kThreads, smem_kv, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  dim3 gq((unsigned)cdiv(p.Sq, attn::bwd::kRows), (unsigned)(p.B * p.Hq));
+  kdq<<<gq, attn::bwd::kThreads, smem_q, st>>>(p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -343,6 +365,59 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
   }
   return D == 64 ? launch_fwd_simt<float, 64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st)
                  : launch_fwd_simt<float, 128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Sk, scale, causal, window, st);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq) {
+  if (B <= 0 || Hq <= 0 || Sq < 0) return 0;
+  return round256((size_t)B * Hq * (size_t)Sq * sizeof(float));
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout, void* dq,
+             void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int window,
+             void* workspace, size_t workspace_bytes, void* stream) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq < 0 || Sk < 0 || window < 0 || !std::isfinite(scale) || !(scale > 0.f))
+    return ATTN_ERR_ARG;
+  if (window > 0 && !causal) return ATTN_ERR_ARG;
+  if (Hq % Hkv) return ATTN_ERR_HEADS;
+  if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > 65535 || (long long)B * Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (Sq > 0 && (!q || !o || !lse || !dout || !dq)) return ATTN_ERR_ARG;
+  if (Sk > 0 && (!k || !v || !dk || !dv)) return ATTN_ERR_ARG;
+  cudaStream_t st = as_stream(stream);
+  const size_t elem = 2;
+  if (Sq == 0 || Sk == 0) {  // no pairs: every gradient is zero
+    if (Sq > 0 && cudaMemsetAsync(dq, 0, (size_t)B * Hq * Sq * D * elem, st) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (Sk > 0 && (cudaMemsetAsync(dk, 0, (size_t)B * Hkv * Sk * D * elem, st) != cudaSuccess ||
+                   cudaMemsetAsync(dv, 0, (size_t)B * Hkv * Sk * D * elem, st) != cudaSuccess))
+      return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
+  for (const void* ptr : {q, k, v, o, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return ATTN_ERR_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      workspace_bytes < attn_bwd_workspace_bytes(B, Hq, Sq))
+    return ATTN_ERR_WORKSPACE;
+  attn::bwd::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<const __nv_bfloat16*>(o);
+  p.lse = lse;
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.delta = static_cast<float*>(workspace);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Sk = Sk;
+  p.scale = scale;
+  p.scale_log2 = scale * attn::kLog2e;
+  p.causal = causal ? 1 : 0;
+  p.window = causal ? window : 0;
+  return D == 64 ? launch_bwd<64>(p, st) : launch_bwd<128>(p, st);
 }
 
 int attn_decode_plan(int B, int Hq, int Hkv, int max_seqlen, int num_sms, int* ctas, int* heads_per_cta) {

@@ -88,6 +88,32 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int window,
                     int dtype, void* stream);
 
+/* ------------------------------------------------------------------ backward
+ * Gradients of attn_fwd / attn_fwd_window with recomputation (CSDN «注意力变体深挖» §6.2,
+ * technique 2, and 追问2/追问3: the backward recomputes the attention matrix from Q, K, V
+ * instead of storing it, so memory stays O(n)).  Given the forward's O and LSE and the
+ * upstream gradient dO:
+ *   P = exp(scale * Q K^T - LSE) on visible pairs (the forward's mask and window),
+ *   dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(dO * O)),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,
+ * with dK and dV of a KV head summed over the Hq/Hkv query heads that share it.
+ *
+ *   q, o, dout, dq  [B, Hq, Sq, D] bf16;  k, v, dk, dv  [B, Hkv, Sk, D] bf16;
+ *   lse             [B, Hq, Sq] fp32, as written by the forward (natural log).
+ * dq, dk, dv are written (not accumulated).  causal and window as in attn_fwd /
+ * attn_fwd_window (window > 0 needs causal).  workspace: device memory of at least
+ * attn_bwd_workspace_bytes(B, Hq, Sq) bytes, 256-byte aligned (it holds rowsum(dO * O));
+ * no initial contents needed.  Products run on the tensor cores in bf16 with fp32
+ * accumulation; P and dS are rounded to bf16 as operands.  D must be 64 or 128; all
+ * pointers 16-byte aligned.  Returns ATTN_OK, ATTN_ERR_ARG, ATTN_ERR_HEADS,
+ * ATTN_ERR_UNSUPPORTED, ATTN_ERR_WORKSPACE or ATTN_ERR_CUDA.
+ */
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Sq);
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv,
+             int B, int Hq, int Hkv, int Sq, int Sk, int D, float scale, int causal, int window,
+             void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------------------ decode
  * Single-token decode against a KV cache (CSDN «注意力变体深挖» §七: each step
  * computes only the new token's Q against the cached K/V; gocoding §5: a paged cache

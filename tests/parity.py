@@ -30,3 +30,23 @@ def compare(o, lse, o_ref, lse_ref, tol, what=""):
     if lse is not None:
         assert stats["lse"] <= tol["lse"], f"{what}: max |dLSE| {stats}"
     return stats
+
+
+# Gradients (bf16 in and out, fp32 accumulation, P and dS rounded to bf16 as MMA operands,
+# O rounded to bf16 by the forward): errors are judged relative to the reference's size.
+GRAD_TOL = dict(max_rel=2e-2, mean_rel=1e-2)
+
+
+def compare_grad(got, ref, tol=GRAD_TOL, what=""):
+    """max|d| / max|ref| and mean|d| / mean|ref| within tolerance."""
+    got = to_f64(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.isfinite(got).all(), f"{what}: non-finite gradient"
+    d = np.abs(got - ref)
+    scale_max = max(float(np.abs(ref).max(initial=0.0)), 1e-30)
+    scale_mean = max(float(np.abs(ref).mean()) if ref.size else 0.0, 1e-30)
+    stats = dict(max_rel=float(d.max(initial=0.0)) / scale_max, mean_rel=(float(d.mean()) if d.size else 0.0) / scale_mean)
+    assert stats["max_rel"] <= tol["max_rel"], f"{what}: {stats}"
+    assert stats["mean_rel"] <= tol["mean_rel"], f"{what}: {stats}"
+    return stats
