@@ -329,6 +329,111 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory");
 }
 
+// End of a segment, once every consumer warp has put its partial for the G heads into the
+// held stage's memory (m_s, l_s: [warps][G] log2-domain max and sum; a_s: [warps][G][D]
+// unnormalised O): merge the warps, write O and LSE (a whole stream) or this CTA's
+// normalised partial (a shared stream), let the CTA that finishes a shared stream last
+// merge all its partials, and release the held stage (empty_held).
+template <int D, int G, int KVB>
+__device__ __forceinline__ void finish_segment(const Params& p, const Segment& sg, float* stage, int h0, int Y,
+                                               long long total, int n, volatile int* last_s, float* lse_f,
+                                               uint32_t empty_held) {
+  constexpr int kCon = kConsumerWarps * 32;
+  const float* m_s = stage;
+  const float* l_s = m_s + kConsumerWarps * G;
+  const float* a_s = l_s + kConsumerWarps * G;
+  const size_t bh0 = (size_t)sg.b * p.Hq + h0;
+  const size_t row = (size_t)blockIdx.x * 2 + (sg.slot > 0 ? 1 : 0);
+  for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
+    const int hh = idx / D, d = idx - hh * D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w4 = 0; w4 < kConsumerWarps; ++w4) M = fmaxf(M, m_s[w4 * G + hh]);
+    float Lsum = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w4 = 0; w4 < kConsumerWarps; ++w4) {
+        const float sc = fast_exp2(m_s[w4 * G + hh] - M);
+        Lsum += l_s[w4 * G + hh] * sc;
+        O += a_s[(w4 * G + hh) * D + d] * sc;
+      }
+    }
+    const float o_val = Lsum > 0.f ? (KVB == 2 ? O / Lsum : O / Lsum * p.v_fac) : 0.f;
+    const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+    if (sg.slot < 0) {  // the whole stream: write the result directly
+      p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);
+      if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_val;
+    } else {
+      p.ws_o[(row * G + hh) * D + d] = o_val;
+      if (d == 0) p.ws_lse[row * G + hh] = lse_val;
+    }
+  }
+
+  if (sg.slot >= 0) {
+    // The last CTA of this stream to finish merges all its partials.
+    __threadfence();
+    consumer_sync<kCon>();
+    int* cnt = p.ws_cnt + (size_t)sg.b * Y + sg.y;
+    if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == sg.nsplit - 1);
+    consumer_sync<kCon>();
+    if (*last_s) {
+      __threadfence();
+      // Partial k of the stream is CTA i0 + k's; only the first of those CTAs can hold the
+      // stream in its second slot (when its range starts before the stream).
+      const int i0 = cta_of(sg.start, total, n);
+      const int slot0 = cta_begin(i0, total, n) >= sg.start ? 0 : 1;
+      const int ns = sg.nsplit;
+      float* w_s = stage;  // [G][kMaxCtas]
+      for (int idx = threadIdx.x; idx < G * ns; idx += kCon) {
+        const int hh = idx / ns, k = idx - hh * ns;
+        const size_t r = (size_t)(i0 + k) * 2 + (k == 0 ? slot0 : 0);
+        w_s[hh * kMaxCtas + k] = __ldcg(p.ws_lse + r * G + hh);
+      }
+      consumer_sync<kCon>();
+      if (threadIdx.x < G) {
+        float* wh = w_s + threadIdx.x * kMaxCtas;
+        float M = -INFINITY;
+        for (int k = 0; k < ns; ++k) M = fmaxf(M, wh[k]);
+        float lse = -INFINITY;
+        if (M != -INFINITY) {
+          float Lsum = 0.f;
+          for (int k = 0; k < ns; ++k) Lsum += expf(wh[k] - M);
+          lse = M + logf(Lsum);
+        }
+        for (int k = 0; k < ns; ++k) wh[k] = lse == -INFINITY ? 0.f : expf(wh[k] - lse);
+        lse_f[threadIdx.x] = lse;
+      }
+      consumer_sync<kCon>();
+      const size_t rstride = (size_t)2 * G * D;  // consecutive CTAs' partials
+      const size_t r0 = (size_t)i0 * 2 + slot0;
+      for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
+        const int hh = idx / D, d = idx - hh * D;
+        const float* wh = w_s + hh * kMaxCtas;
+        // partial 0 sits in row r0; partial k >= 1 in row 2 * (i0 + k)
+        float out0 = wh[0] * __ldcg(p.ws_o + (r0 * G + hh) * D + d);
+        float out1 = 0.f, out2 = 0.f, out3 = 0.f;
+        const float* o_s = p.ws_o + ((size_t)i0 * 2 * G + hh) * D + d;
+        int k = 1;
+        for (; k + 3 <= ns; k += 3) {
+          out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
+          out2 = fmaf(wh[k + 1], __ldcg(o_s + (k + 1) * rstride), out2);
+          out3 = fmaf(wh[k + 2], __ldcg(o_s + (k + 2) * rstride), out3);
+        }
+        for (; k < ns; ++k) out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
+        p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
+        if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
+      }
+      if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
+    }
+  }
+  // Release the held stage once every consumer is done with its memory; the proxy fence
+  // orders this CTA's generic writes to it before the copies that will refill it.
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  consumer_sync<kCon>();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(empty_held);
+}
+
 template <int D, int G, int KVB>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   // Lanes per token row: 8, except D=128 with 8 heads per CTA, where 16 lanes halve the
@@ -661,94 +766,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
     }
     consumer_sync<kCon>();
     if (!*ok_s) return;
-    const size_t bh0 = (size_t)sg.b * p.Hq + h0;
-    const size_t row = (size_t)blockIdx.x * 2 + (sg.slot > 0 ? 1 : 0);
-    for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
-      const int hh = idx / D, d = idx - hh * D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w4 = 0; w4 < kConsumerWarps; ++w4) M = fmaxf(M, m_s[w4 * G + hh]);
-      float Lsum = 0.f, O = 0.f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w4 = 0; w4 < kConsumerWarps; ++w4) {
-          const float sc = fast_exp2(m_s[w4 * G + hh] - M);
-          Lsum += l_s[w4 * G + hh] * sc;
-          O += a_s[(w4 * G + hh) * D + d] * sc;
-        }
-      }
-      const float o_val = Lsum > 0.f ? (KVB == 2 ? O / Lsum : O / Lsum * p.v_fac) : 0.f;
-      const float lse_val = Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
-      if (sg.slot < 0) {  // the whole stream: write the result directly
-        p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(o_val);
-        if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_val;
-      } else {
-        p.ws_o[(row * G + hh) * D + d] = o_val;
-        if (d == 0) p.ws_lse[row * G + hh] = lse_val;
-      }
-    }
-
-    if (sg.slot >= 0) {
-      // The last CTA of this stream to finish merges all its partials.
-      __threadfence();
-      consumer_sync<kCon>();
-      int* cnt = p.ws_cnt + (size_t)sg.b * Y + sg.y;
-      if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == sg.nsplit - 1);
-      consumer_sync<kCon>();
-      if (*last_s) {
-        __threadfence();
-        // Partial k of the stream is CTA i0 + k's; only the first of those CTAs can hold the
-        // stream in its second slot (when its range starts before the stream).
-        const int i0 = cta_of(sg.start, total, n);
-        const int slot0 = cta_begin(i0, total, n) >= sg.start ? 0 : 1;
-        const int ns = sg.nsplit;
-        float* w_s = reinterpret_cast<float*>(smem + held * L::kSlotBytes);  // [G][kMaxCtas]
-        for (int idx = threadIdx.x; idx < G * ns; idx += kCon) {
-          const int hh = idx / ns, k = idx - hh * ns;
-          const size_t r = (size_t)(i0 + k) * 2 + (k == 0 ? slot0 : 0);
-          w_s[hh * kMaxCtas + k] = __ldcg(p.ws_lse + r * G + hh);
-        }
-        consumer_sync<kCon>();
-        if (threadIdx.x < G) {
-          float* wh = w_s + threadIdx.x * kMaxCtas;
-          float M = -INFINITY;
-          for (int k = 0; k < ns; ++k) M = fmaxf(M, wh[k]);
-          float lse = -INFINITY;
-          if (M != -INFINITY) {
-            float Lsum = 0.f;
-            for (int k = 0; k < ns; ++k) Lsum += expf(wh[k] - M);
-            lse = M + logf(Lsum);
-          }
-          for (int k = 0; k < ns; ++k) wh[k] = lse == -INFINITY ? 0.f : expf(wh[k] - lse);
-          lse_f[threadIdx.x] = lse;
-        }
-        consumer_sync<kCon>();
-        const size_t rstride = (size_t)2 * G * D;  // consecutive CTAs' partials
-        const size_t r0 = (size_t)i0 * 2 + slot0;
-        for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
-          const int hh = idx / D, d = idx - hh * D;
-          const float* wh = w_s + hh * kMaxCtas;
-          // partial 0 sits in row r0; partial k >= 1 in row 2 * (i0 + k)
-          float out0 = wh[0] * __ldcg(p.ws_o + (r0 * G + hh) * D + d);
-          float out1 = 0.f, out2 = 0.f, out3 = 0.f;
-          const float* o_s = p.ws_o + ((size_t)i0 * 2 * G + hh) * D + d;
-          int k = 1;
-          for (; k + 3 <= ns; k += 3) {
-            out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
-            out2 = fmaf(wh[k + 1], __ldcg(o_s + (k + 1) * rstride), out2);
-            out3 = fmaf(wh[k + 2], __ldcg(o_s + (k + 2) * rstride), out3);
-          }
-          for (; k < ns; ++k) out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
-          p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
-          if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
-        }
-        if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
-      }
-    }
-    // Release the held stage once every consumer is done with its memory.
-    consumer_sync<kCon>();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty_bar(held));
+    finish_segment<D, G, KVB>(p, sg, reinterpret_cast<float*>(smem + held * L::kSlotBytes), h0, Y, total, n, last_s,
+                              lse_f, empty_bar(held));
   }
 }
 

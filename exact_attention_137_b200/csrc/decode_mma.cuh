@@ -1,0 +1,373 @@
+// Single-token decode with the consumers on the warp-level tensor cores, for bf16 caches
+// whose rows come in runs of 16 tokens: a dense cache, or a paged pool whose page size is a
+// multiple of 16 (gocoding §5's fixed-size blocks).
+//
+// The schedule, the segments, the split-KV partials and their merge are those of
+// decode_kernel (decode.cuh): only the stage layout and the consumers differ.
+//
+//  * Stages hold 64 consecutive tokens of a segment, starting at a multiple of 16 in the
+//    sequence: four 16-token granules, each one page-aligned run of rows.  warp 4 moves each
+//    granule's K and V with 3-D TMA loads (64-column boxes, 128-byte swizzle) from the pool
+//    viewed as (D, rows of a block, block * Hkv + kv head).  Granules past the segment are
+//    not loaded; tokens of a granule outside the segment are masked.
+//  * Consumer warp w owns granule w of every stage.  With the G query heads of the segment
+//    as the N = 8 side of m16n8k16 MMAs (bf16 in, fp32 accumulate):
+//        S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8)          D/16 MMAs
+//        O^T (D x 8 heads)        += V^T (D x 16 tokens) . P^T (16 x 8)  D/16 MMAs
+//    K comes from ldmatrix, V from ldmatrix.trans (the swizzle keeps both conflict-free),
+//    and P^T's fragment is the score fragment rounded to bf16 and transposed in registers
+//    (movmatrix).  Each lane holds the scores of two heads for two tokens; a head's max
+//    over the granule takes three shuffles.  The online softmax per head is that of the
+//    pages (CSDN «注意力变体深挖» §6.2: running max, rescale by exp(m_old - m_new)), in
+//    the log2 domain; l sums the fp32 probabilities, P enters the MMA rounded to bf16.
+//  * About 7 warp instructions per token and KV head, against about 50 for the fp32 FFMA
+//    consumers of decode_kernel, whose issue rate bounded them.
+#pragma once
+
+#include <cuda.h>
+
+#include "decode.cuh"
+
+namespace attn {
+namespace dec {
+
+constexpr int kGranule = 16;  // tokens per consumer warp and stage
+static_assert(kGranule * kConsumerWarps == kStageTokens, "one granule per consumer warp");
+
+template <int D, int G>
+struct MmaLayout {
+  static constexpr int kHalves = D / 64;                     // 128-byte swizzled column halves of a row
+  static constexpr int kHalfBytes = kStageTokens * 128;      // one half of a stage's K (or V)
+  static constexpr int kGranHalfBytes = kGranule * 128;      // one half of one granule
+  static constexpr int kStageBytes = kHalves * kHalfBytes;   // K (or V) of one stage
+  static constexpr int kSlotBytes = 2 * kStageBytes;         // K, then V
+  static constexpr int kGranTx = 2 * kHalves * kGranHalfBytes;  // bytes a granule's loads deliver
+  static constexpr int kQRow = D * 2;
+  static constexpr int kQBytes = G * kQRow;
+  static constexpr int kQ = kStages * kSlotBytes;
+  static constexpr int kBar = kQ + kStages * kQBytes;
+  static constexpr int kMisc = kBar + 2 * kStages * 8;
+  static constexpr int kSeg = kMisc + 64;
+  static constexpr int kBytes = kSeg + 128;
+  static constexpr int kAlloc = kBytes + 1024;  // the base is aligned up to 1024 bytes (swizzle atom)
+  static_assert(kSlotBytes % 1024 == 0 && kBar % 8 == 0, "stage alignment");
+  static_assert(4 * (2 * kConsumerWarps * G + kConsumerWarps * G * D) <= kSlotBytes, "warp merge fits a stage");
+  static_assert(4 * G * kMaxCtas <= kSlotBytes, "merge weights fit a stage");
+  static_assert(sizeof(SegSlots) <= kBytes - kSeg, "segment slots fit");
+};
+
+// Byte offset of 16-byte chunk c (0 .. D/8-1) of row r in a stage's K or V: the row's two
+// 64-column halves live in separate 128-byte-swizzled blocks of 64 rows.
+template <int D>
+__device__ __forceinline__ uint32_t sw_off(int r, int c) {
+  return (uint32_t)((c >> 3) * (kStageTokens * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ float shfl_max_rows(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+}
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const Params p) {
+  static_assert(G >= 1 && G <= 8, "the heads are the N = 8 side of the MMA");
+  static_assert(D == 64 || D == 128, "head dim");
+  using L = MmaLayout<D, G>;
+  constexpr int KS = D / 16;  // k-steps of S^T and m-tiles of O^T
+
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  auto full_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * s; };
+  auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (kStages + s); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
+  volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
+  float* lse_f = reinterpret_cast<float*>(smem + L::kMisc + 32);  // [G]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int Y = p.Hkv * p.nsub;
+  const int g = p.Hq / p.Hkv;
+  const long long total = total_units(p, Y, lane, blockIdx.x == 0 && warp == 0);
+
+  // Empty sequences have no units; CTA i writes O = 0, LSE = -inf for b = i mod grid.
+  if (warp < kConsumerWarps) {
+    for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+      if (checked_len(p, b, false) != 0) continue;
+      for (int idx = threadIdx.x; idx < p.Hq * D; idx += kConsumerWarps * 32) {
+        p.o[(size_t)b * p.Hq * D + idx] = __float2bfloat16_rn(0.f);
+        if (p.lse != nullptr && idx % D == 0) p.lse[(size_t)b * p.Hq + idx / D] = -INFINITY;
+      }
+    }
+  }
+  const int n = active_ctas(total, gridDim.x);
+  if ((int)blockIdx.x >= n) return;
+  auto len_of = [&](int b) -> int { return span_len(p, b, false); };
+  // Absolute cache positions of a segment: tokens count from the first attended one, which
+  // sits at `base` in the cache; stages start at the multiple of 16 at or below the first.
+  auto seg_base = [&](const Segment& sg) -> int {
+    return p.window > 0 ? checked_len(p, sg.b, false) - len_of(sg.b) : 0;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  Walk w = walk_start(p, Y, total, n, blockIdx.x, lane);
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+    }
+    const int bs = p.block_size;
+    const bool paged = p.block_table != nullptr;
+    int last_fill[kStages];
+    for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+    int it = 0;
+    bool alive = true;
+    Segment sg;
+    while (alive && next_segment(w, len_of, Y, total, n, sg)) {
+      const int kvh = sg.y / p.nsub;
+      const int h0 = kvh * g + (sg.y - kvh * p.nsub) * G;
+      const int* table = paged ? p.block_table + (size_t)sg.b * p.max_blocks : nullptr;
+      auto load_id = [&](int page) -> int {
+        return (paged && page < p.max_blocks) ? __ldg(table + page) : -1;
+      };
+      const int base = seg_base(sg);
+      const int lo = base + sg.tok0, hi = base + sg.tok1;
+      const int a0 = lo & ~(kGranule - 1);
+      const int nst = (hi - a0 + kStageTokens - 1) / kStageTokens;
+      int cur_first = a0 / bs;
+      int nxt_first = cur_first + 32;
+      int cur_id = load_id(cur_first + lane);
+      int nxt_id = load_id(nxt_first + lane);
+      for (int st = 0; st < nst; ++st, ++it) {
+        const int s = it % kStages;
+        const int f = it / kStages;
+        if (f > 0) {
+          alive = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), (f - 1) & 1, abort_flag));
+          if (!alive) break;
+        }
+        const uint32_t dk = sbase + s * L::kSlotBytes;
+        const uint32_t dv = dk + L::kStageBytes;
+        if (st == 0 && lane == 0) {
+          mbar_expect_tx(full_bar(s), (uint32_t)L::kQBytes);
+          bulk_load(sbase + L::kQ + s * L::kQBytes, p.q + ((size_t)sg.b * p.Hq + h0) * D, (uint32_t)L::kQBytes,
+                    full_bar(s));
+        }
+        for (int q = 0; q < kConsumerWarps; ++q) {
+          const int a = a0 + st * kStageTokens + q * kGranule;  // the granule's first position
+          if (a >= hi) break;
+          const int page = a / bs;
+          const int slot = a - page * bs;
+          while (page >= cur_first + 32) {
+            cur_id = nxt_id;
+            cur_first = nxt_first;
+            nxt_first += 32;
+            nxt_id = load_id(nxt_first + lane);
+          }
+          const int blk = paged ? __shfl_sync(0xffffffffu, cur_id, page - cur_first) : sg.b;
+          if (lane == 0) {
+            if (blk < 0 || blk >= p.num_blocks) {
+              flag_error(p, ATTN_DEV_BAD_BLOCK);
+            } else {
+              const int z = blk * p.Hkv + kvh;
+              mbar_expect_tx(full_bar(s), (uint32_t)L::kGranTx);
+#pragma unroll
+              for (int hf = 0; hf < L::kHalves; ++hf) {
+                const uint32_t off = hf * L::kHalfBytes + q * L::kGranHalfBytes;
+                tma_load_3d(dk + off, &tmK, full_bar(s), 64 * hf, slot, z);
+                tma_load_3d(dv + off, &tmV, full_bar(s), 64 * hf, slot, z);
+              }
+            }
+          }
+        }
+        if (lane == 0) mbar_arrive(full_bar(s));
+        last_fill[s] = f;
+      }
+    }
+    if (*abort_flag && lane == 0) {
+      // Consumers gave up: let copies already in flight land before the CTA exits.
+      int never = 0;
+      for (int s = 0; s < kStages; ++s)
+        if (last_fill[s] >= 0) mbar_wait(full_bar(s), last_fill[s] & 1, &never, 100000000ull);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  constexpr int kCon = kConsumerWarps * 32;
+  const int g8 = lane >> 2, t4 = lane & 3;  // fragment row group and column pair
+  const float c = p.scale_log2;
+  SegSlots* ss = reinterpret_cast<SegSlots*>(smem + L::kSeg);
+  volatile int* has = ss->has;
+  if (threadIdx.x == 0) {
+    has[0] = next_segment(w, len_of, Y, total, n, ss->sg[0]);
+    ss->w = w;
+  }
+  consumer_sync<kCon>();
+  // ldmatrix rows of this warp's granule.  K, the row-major A of S^T: lane l addresses token
+  // 8 * ((l >> 3) & 1) + (l & 7), chunk 2 * ks + (l >> 4).  V, read transposed as the A of
+  // O^T: token 8 * (l >> 4) + (l & 7), chunk 2 * mt + ((l >> 3) & 1).
+  const int rk = warp * kGranule + ((lane >> 3) & 1) * 8 + (lane & 7);
+  const int ck = lane >> 4;
+  const int rv = warp * kGranule + (lane >> 4) * 8 + (lane & 7);
+  const int cv = (lane >> 3) & 1;
+  int it = 0;
+  for (int k = 0; has[k & 1]; ++k) {
+    if (threadIdx.x == 0) {  // one segment ahead, into the other slot
+      Walk wn = ss->w;
+      has[(k + 1) & 1] = next_segment(wn, len_of, Y, total, n, ss->sg[(k + 1) & 1]);
+      ss->w = wn;
+    }
+    const Segment& sg = ss->sg[k & 1];
+    const int kvh = sg.y / p.nsub;
+    const int h0 = kvh * g + (sg.y - kvh * p.nsub) * G;
+    const int base = seg_base(sg);
+    const int lo = base + sg.tok0, hi = base + sg.tok1;
+    const int a0 = lo & ~(kGranule - 1);
+    const int nst = (hi - a0 + kStageTokens - 1) / kStageTokens;
+    uint32_t qf[KS][2];  // B fragments of Q^T (k = dims, n = heads); heads >= G are zero
+    float acc[KS][4];    // O^T tiles: rows = dims 16 mt + g8 (+8), columns = heads 2 t4, 2 t4 + 1
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2 t4 and 2 t4 + 1
+
+    bool ok = true;
+    int held = 0;
+    for (int st = 0; st < nst; ++st) {
+      const int s = it % kStages;
+      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / kStages) & 1, abort_flag));
+      if (!ok) break;
+      ++it;
+      held = s;
+      if (st == 0) {
+        const uint8_t* sq = smem + L::kQ + s * L::kQBytes + g8 * L::kQRow;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          qf[ks][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 2 * t4) * 2) : 0u;
+          qf[ks][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 8 + 2 * t4) * 2) : 0u;
+        }
+      }
+      const int a = a0 + st * kStageTokens + warp * kGranule;  // this warp's granule
+      if (a < hi) {
+        const uint32_t sk = sbase + s * L::kSlotBytes;
+        const uint32_t sv = sk + L::kStageBytes;
+        // S^T = K Q^T, the k-steps alternating between two accumulators.
+        float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t af[4];
+          ldsm_x4(sk + sw_off<D>(rk, 2 * ks + ck), af[0], af[1], af[2], af[3]);
+          if (ks & 1) mma16816(so, af, qf[ks][0], qf[ks][1]);
+          else mma16816(se, af, qf[ks][0], qf[ks][1]);
+        }
+        // x[0], x[1]: token g8, heads 2 t4, 2 t4 + 1; x[2], x[3]: token g8 + 8.
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) x[e] = (se[e] + so[e]) * c;
+        const bool edge = a < lo || a + kGranule > hi;  // warp-uniform
+        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;    // V fragment masks (tokens 2 t4 .., 2 t4 + 8 ..)
+        if (edge) {
+          const int ta = a + g8, tb = ta + 8;
+          if (!(ta >= lo && ta < hi)) x[0] = x[1] = -INFINITY;
+          if (!(tb >= lo && tb < hi)) x[2] = x[3] = -INFINITY;
+          const int t0 = a + 2 * t4;
+          mlo = (t0 >= lo && t0 < hi ? 0x0000ffffu : 0u) | (t0 + 1 >= lo && t0 + 1 < hi ? 0xffff0000u : 0u);
+          mhi = (t0 + 8 >= lo && t0 + 8 < hi ? 0x0000ffffu : 0u) | (t0 + 9 >= lo && t0 + 9 < hi ? 0xffff0000u : 0u);
+        }
+        // Online softmax per head; every granule holds an attended token, so the new max is
+        // finite and the first rescale factor is exp2(-inf) = 0.
+        const float n0 = fmaxf(m0, shfl_max_rows(fmaxf(x[0], x[2])));
+        const float n1 = fmaxf(m1, shfl_max_rows(fmaxf(x[1], x[3])));
+        const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
+        m0 = n0;
+        m1 = n1;
+        const float p0 = fast_exp2(x[0] - n0), p1 = fast_exp2(x[1] - n1);
+        const float p2 = fast_exp2(x[2] - n0), p3 = fast_exp2(x[3] - n1);
+        l0 = fmaf(l0, al0, p0 + p2);
+        l1 = fmaf(l1, al1, p1 + p3);
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            acc[mt][0] *= al0;
+            acc[mt][1] *= al1;
+            acc[mt][2] *= al0;
+            acc[mt][3] *= al1;
+          }
+        }
+        // P^T's B fragment: lane (g8, t4) needs P[tokens 2 t4, 2 t4 + 1 (+8)][head g8].
+        const uint32_t b0 = movmatrix_t(pack_bf16x2(p0, p1));
+        const uint32_t b1 = movmatrix_t(pack_bf16x2(p2, p3));
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          uint32_t af[4];
+          ldsm_x4_t(sv + sw_off<D>(rv, 2 * mt + cv), af[0], af[1], af[2], af[3]);
+          af[0] &= mlo;
+          af[1] &= mlo;
+          af[2] &= mhi;
+          af[3] &= mhi;
+          mma16816(acc[mt], af, b0, b1);
+        }
+      }
+      if (st + 1 < nst) {  // the segment's last stage stays held for the merge below
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty_bar(s));
+      }
+    }
+
+    // ------------------------------------------------ end of segment: merge the warps
+    consumer_sync<kCon>();
+    float* m_s = reinterpret_cast<float*>(smem + held * L::kSlotBytes);  // [warps][G]
+    float* l_s = m_s + kConsumerWarps * G;                                // [warps][G]
+    float* a_s = l_s + kConsumerWarps * G;                                // [warps][G][D]
+    if (threadIdx.x == 0) *ok_s = (*abort_flag == 0);
+    if (ok) {
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+      }
+      const int hA = 2 * t4, hB = hA + 1;
+      if (g8 == 0) {
+        if (hA < G) {
+          m_s[warp * G + hA] = m0;
+          l_s[warp * G + hA] = l0;
+        }
+        if (hB < G) {
+          m_s[warp * G + hB] = m1;
+          l_s[warp * G + hB] = l1;
+        }
+      }
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        const int d = 16 * mt + g8;
+        if (hA < G) {
+          a_s[(warp * G + hA) * D + d] = acc[mt][0];
+          a_s[(warp * G + hA) * D + d + 8] = acc[mt][2];
+        }
+        if (hB < G) {
+          a_s[(warp * G + hB) * D + d] = acc[mt][1];
+          a_s[(warp * G + hB) * D + d + 8] = acc[mt][3];
+        }
+      }
+    }
+    consumer_sync<kCon>();
+    if (!*ok_s) return;
+    finish_segment<D, G, 2>(p, sg, m_s, h0, Y, total, n, last_s, lse_f, empty_bar(held));
+  }
+}
+
+}  // namespace dec
+}  // namespace attn
