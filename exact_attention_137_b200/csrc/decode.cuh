@@ -196,9 +196,8 @@ struct Layout {
   static constexpr int kMisc = kBar + 2 * kStages * 8;
   static constexpr int kSeg = kMisc + 64;  // consumers' walk state and two segment slots
   static constexpr int kBytes = kSeg + 128;
-  // The end-of-segment merge and the cross-CTA merge run in the held stage's memory.
+  // The end-of-segment merge of the warps runs in the held stage's memory.
   static_assert(4 * (2 * kConsumerWarps * G + kConsumerWarps * G * D) <= kSlotBytes, "warp merge fits a stage");
-  static_assert(4 * G * kMaxCtas <= kSlotBytes, "merge weights fit a stage");
   static_assert(sizeof(SegSlots) <= kBytes - kSeg, "segment slots fit");
 };
 
@@ -255,20 +254,27 @@ __device__ __forceinline__ long long shfl_up_ll(long long v, int d) {
   return ((long long)hi << 32) | (unsigned int)lo;
 }
 
-// Units over all streams; every lane of the warp returns the same value.
-__device__ __forceinline__ long long total_units(const Params& p, int Y, int lane, bool report) {
+// Units over all streams, lenf(b) being the attended length of sequence b (it is called
+// with b = b0 + lane, b0 = 0, 32, ..., and returns 0 for b >= B); every lane of the warp
+// returns the same value.
+template <class LenF>
+__device__ __forceinline__ long long total_units_of(const Params& p, int Y, int lane, const LenF& lenf) {
   long long sum = 0;
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int b = b0 + lane;
-    sum += b < p.B ? units_of(span_len(p, b, report)) : 0;
-  }
+  for (int b0 = 0; b0 < p.B; b0 += 32) sum += units_of(lenf(b0 + lane));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += shfl_ll(sum, lane ^ o);
   return sum * Y;
 }
 
-// walk_start_host with a warp: a prefix scan over the sequences, 32 at a time.
-__device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long total, int n, int i, int lane) {
+__device__ __forceinline__ long long total_units(const Params& p, int Y, int lane, bool report) {
+  return total_units_of(p, Y, lane, [&](int b) { return b < p.B ? span_len(p, b, report) : 0; });
+}
+
+// walk_start_host with a warp: a prefix scan over the sequences, 32 at a time (lenf as in
+// total_units_of).
+template <class LenF>
+__device__ __forceinline__ Walk walk_start_of(const Params& p, int Y, long long total, int n, int i, int lane,
+                                              const LenF& lenf) {
   Walk w;
   w.pos = cta_begin(i, total, n);
   w.hi = cta_begin(i + 1, total, n);
@@ -281,7 +287,7 @@ __device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long tot
   long long prefix = 0;
   for (int b0 = 0; b0 < p.B; b0 += 32) {
     const int b = b0 + lane;
-    const int len = b < p.B ? span_len(p, b, false) : 0;
+    const int len = lenf(b);
     const long long span = (long long)Y * units_of(len);
     long long incl = span;
 #pragma unroll
@@ -304,6 +310,10 @@ __device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long tot
   }
   w.hi = w.pos;
   return w;
+}
+
+__device__ __forceinline__ Walk walk_start(const Params& p, int Y, long long total, int n, int i, int lane) {
+  return walk_start_of(p, Y, total, n, i, lane, [&](int b) { return b < p.B ? span_len(p, b, false) : 0; });
 }
 
 // Recursive-halving reduce-scatter over the LPT lanes of a group: on return lane j of
@@ -329,15 +339,12 @@ __device__ __forceinline__ void consumer_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kCount) : "memory");
 }
 
-// End of a segment, once every consumer warp has put its partial for the G heads into the
-// held stage's memory (m_s, l_s: [warps][G] log2-domain max and sum; a_s: [warps][G][D]
-// unnormalised O): merge the warps, write O and LSE (a whole stream) or this CTA's
-// normalised partial (a shared stream), let the CTA that finishes a shared stream last
-// merge all its partials, and release the held stage (empty_held).
+// End of a segment, part 1, once every consumer warp has put its partial for the G heads
+// into the held stage's memory (m_s, l_s: [warps][G] log2-domain max and sum; a_s:
+// [warps][G][D] unnormalised O): merge the warps and write O and LSE (a whole stream) or
+// this CTA's normalised partial (a shared stream).
 template <int D, int G, int KVB>
-__device__ __forceinline__ void finish_segment(const Params& p, const Segment& sg, float* stage, int h0, int Y,
-                                               long long total, int n, volatile int* last_s, float* lse_f,
-                                               uint32_t empty_held) {
+__device__ __forceinline__ void write_segment(const Params& p, const Segment& sg, const float* stage, int h0) {
   constexpr int kCon = kConsumerWarps * 32;
   const float* m_s = stage;
   const float* l_s = m_s + kConsumerWarps * G;
@@ -368,64 +375,71 @@ __device__ __forceinline__ void finish_segment(const Params& p, const Segment& s
       if (d == 0) p.ws_lse[row * G + hh] = lse_val;
     }
   }
+}
 
-  if (sg.slot >= 0) {
-    // The last CTA of this stream to finish merges all its partials.
-    __threadfence();
-    consumer_sync<kCon>();
-    int* cnt = p.ws_cnt + (size_t)sg.b * Y + sg.y;
-    if (threadIdx.x == 0) *last_s = (atomicAdd(cnt, 1) == sg.nsplit - 1);
-    consumer_sync<kCon>();
-    if (*last_s) {
-      __threadfence();
-      // Partial k of the stream is CTA i0 + k's; only the first of those CTAs can hold the
-      // stream in its second slot (when its range starts before the stream).
-      const int i0 = cta_of(sg.start, total, n);
-      const int slot0 = cta_begin(i0, total, n) >= sg.start ? 0 : 1;
-      const int ns = sg.nsplit;
-      float* w_s = stage;  // [G][kMaxCtas]
-      for (int idx = threadIdx.x; idx < G * ns; idx += kCon) {
-        const int hh = idx / ns, k = idx - hh * ns;
-        const size_t r = (size_t)(i0 + k) * 2 + (k == 0 ? slot0 : 0);
-        w_s[hh * kMaxCtas + k] = __ldcg(p.ws_lse + r * G + hh);
-      }
-      consumer_sync<kCon>();
-      if (threadIdx.x < G) {
-        float* wh = w_s + threadIdx.x * kMaxCtas;
-        float M = -INFINITY;
-        for (int k = 0; k < ns; ++k) M = fmaxf(M, wh[k]);
-        float lse = -INFINITY;
-        if (M != -INFINITY) {
-          float Lsum = 0.f;
-          for (int k = 0; k < ns; ++k) Lsum += expf(wh[k] - M);
-          lse = M + logf(Lsum);
-        }
-        for (int k = 0; k < ns; ++k) wh[k] = lse == -INFINITY ? 0.f : expf(wh[k] - lse);
-        lse_f[threadIdx.x] = lse;
-      }
-      consumer_sync<kCon>();
-      const size_t rstride = (size_t)2 * G * D;  // consecutive CTAs' partials
-      const size_t r0 = (size_t)i0 * 2 + slot0;
-      for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
-        const int hh = idx / D, d = idx - hh * D;
-        const float* wh = w_s + hh * kMaxCtas;
-        // partial 0 sits in row r0; partial k >= 1 in row 2 * (i0 + k)
-        float out0 = wh[0] * __ldcg(p.ws_o + (r0 * G + hh) * D + d);
-        float out1 = 0.f, out2 = 0.f, out3 = 0.f;
-        const float* o_s = p.ws_o + ((size_t)i0 * 2 * G + hh) * D + d;
-        int k = 1;
-        for (; k + 3 <= ns; k += 3) {
-          out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
-          out2 = fmaf(wh[k + 1], __ldcg(o_s + (k + 1) * rstride), out2);
-          out3 = fmaf(wh[k + 2], __ldcg(o_s + (k + 2) * rstride), out3);
-        }
-        for (; k < ns; ++k) out1 = fmaf(wh[k], __ldcg(o_s + k * rstride), out1);
-        p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn((out0 + out1) + (out2 + out3));
-        if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = lse_f[hh];
-      }
-      if (threadIdx.x == 0) *cnt = 0;  // ready for the next call
+// The merge of a shared stream's nsplit partials (O_s normalised, lse_s natural log), by the
+// CTA that counted the stream last: LSE = log sum_s exp(lse_s), O = sum_s exp(lse_s - LSE) O_s,
+// the pages' two-way online-softmax merge applied across CTAs, here as a running merge so
+// that all the loads of a thread are independent of one another.
+template <int D, int G>
+__device__ __forceinline__ void merge_stream(const Params& p, const Segment& sg, int h0, long long total, int n) {
+  constexpr int kCon = kConsumerWarps * 32;
+  const size_t bh0 = (size_t)sg.b * p.Hq + h0;
+  // Partial k of the stream is CTA i0 + k's; only the first of those CTAs can hold the
+  // stream in its second slot (when its range starts before the stream).
+  const int i0 = cta_of(sg.start, total, n);
+  const int slot0 = cta_begin(i0, total, n) >= sg.start ? 0 : 1;
+  const int ns = sg.nsplit;
+  for (int idx = threadIdx.x; idx < G * D; idx += kCon) {
+    const int hh = idx / D, d = idx - hh * D;
+    float M = -INFINITY, Lw = 0.f, acc = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < ns; ++k) {
+      const size_t r = (size_t)(i0 + k) * 2 + (k == 0 ? slot0 : 0);
+      const float lk = __ldcg(p.ws_lse + r * G + hh);
+      const float ok = __ldcg(p.ws_o + (r * G + hh) * D + d);
+      const float mn = fmaxf(M, lk);
+      const float s1 = mn == -INFINITY ? 0.f : expf(M - mn);
+      const float s2 = mn == -INFINITY ? 0.f : expf(lk - mn);
+      Lw = fmaf(Lw, s1, s2);
+      acc = fmaf(acc, s1, s2 * ok);
+      M = mn;
     }
+    p.o[(bh0 + hh) * D + d] = __float2bfloat16_rn(Lw > 0.f ? acc / Lw : 0.f);
+    if (p.lse != nullptr && d == 0) p.lse[bh0 + hh] = Lw > 0.f ? M + logf(Lw) : -INFINITY;
   }
+}
+
+// Count this CTA's partial of a shared stream, after a barrier that follows the CTA's partial
+// writes; true for the CTA that counts last (it also returns the counter to zero, since every
+// other CTA of the stream has counted, ready for the next call).
+__device__ __forceinline__ bool count_partial(const Params& p, const Segment& sg, int Y) {
+  int* cnt = p.ws_cnt + (size_t)sg.b * Y + sg.y;
+  const bool last = atom_add_acq_rel_gpu(cnt, 1) == sg.nsplit - 1;
+  if (last) *cnt = 0;
+  return last;
+}
+
+// Part 2, for a shared stream whose partial this CTA has written: count it, and if this CTA
+// is the stream's last, merge its partials.
+template <int D, int G>
+__device__ __forceinline__ void complete_stream(const Params& p, const Segment& sg, int h0, int Y, long long total,
+                                                int n, volatile int* last_s) {
+  constexpr int kCon = kConsumerWarps * 32;
+  consumer_sync<kCon>();
+  if (threadIdx.x == 0) *last_s = count_partial(p, sg, Y);
+  consumer_sync<kCon>();
+  if (*last_s) merge_stream<D, G>(p, sg, h0, total, n);
+}
+
+// Both parts, then the release of the held stage (empty_held).
+template <int D, int G, int KVB>
+__device__ __forceinline__ void finish_segment(const Params& p, const Segment& sg, float* stage, int h0, int Y,
+                                               long long total, int n, volatile int* last_s,
+                                               uint32_t empty_held) {
+  constexpr int kCon = kConsumerWarps * 32;
+  write_segment<D, G, KVB>(p, sg, stage, h0);
+  if (sg.slot >= 0) complete_stream<D, G>(p, sg, h0, Y, total, n, last_s);
   // Release the held stage once every consumer is done with its memory; the proxy fence
   // orders this CTA's generic writes to it before the copies that will refill it.
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -484,7 +498,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
   volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  float* lse_f = reinterpret_cast<float*>(smem + L::kMisc + 32);  // [G]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Y = p.Hkv * p.nsub;
@@ -767,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const Params p) {
     consumer_sync<kCon>();
     if (!*ok_s) return;
     finish_segment<D, G, KVB>(p, sg, reinterpret_cast<float*>(smem + held * L::kSlotBytes), h0, Y, total, n, last_s,
-                              lse_f, empty_bar(held));
+                              empty_bar(held));
   }
 }
 

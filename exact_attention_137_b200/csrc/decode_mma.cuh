@@ -52,7 +52,6 @@ struct MmaLayout {
   static constexpr int kAlloc = kBytes + 1024;  // the base is aligned up to 1024 bytes (swizzle atom)
   static_assert(kSlotBytes % 1024 == 0 && kBar % 8 == 0, "stage alignment");
   static_assert(4 * (2 * kConsumerWarps * G + kConsumerWarps * G * D) <= kSlotBytes, "warp merge fits a stage");
-  static_assert(4 * G * kMaxCtas <= kSlotBytes, "merge weights fit a stage");
   static_assert(sizeof(SegSlots) <= kBytes - kSeg, "segment slots fit");
 };
 
@@ -86,18 +85,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (kStages + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
   volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
-  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);
-  float* lse_f = reinterpret_cast<float*>(smem + L::kMisc + 32);  // [G]
+  volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int Y = p.Hkv * p.nsub;
   const int g = p.Hq / p.Hkv;
-  const long long total = total_units(p, Y, lane, blockIdx.x == 0 && warp == 0);
+  // With at most 32 sequences each lane loads one length once, and the schedule below is
+  // computed from registers (one global round trip before the first copy).
+  const bool few = p.B <= 32;
+  const int len_l = few && lane < p.B ? span_len(p, lane, blockIdx.x == 0 && warp == 0) : 0;
+  auto lenf = [&](int b) -> int { return few ? len_l : (b < p.B ? span_len(p, b, false) : 0); };
+  const long long total = few ? total_units_of(p, Y, lane, lenf) : total_units(p, Y, lane, blockIdx.x == 0 && warp == 0);
 
   // Empty sequences have no units; CTA i writes O = 0, LSE = -inf for b = i mod grid.
   if (warp < kConsumerWarps) {
     for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-      if (checked_len(p, b, false) != 0) continue;
+      if ((few ? __shfl_sync(0xffffffffu, len_l, b) : checked_len(p, b, false)) != 0) continue;
       for (int idx = threadIdx.x; idx < p.Hq * D; idx += kConsumerWarps * 32) {
         p.o[(size_t)b * p.Hq * D + idx] = __float2bfloat16_rn(0.f);
         if (p.lse != nullptr && idx % D == 0) p.lse[(size_t)b * p.Hq + idx / D] = -INFINITY;
@@ -122,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     fence_barrier_init();
   }
   __syncthreads();
-  Walk w = walk_start(p, Y, total, n, blockIdx.x, lane);
+  Walk w = walk_start_of(p, Y, total, n, blockIdx.x, lane, lenf);
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ TMA producer
@@ -224,6 +227,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int ck = lane >> 4;
   const int rv = warp * kGranule + (lane >> 4) * 8 + (lane & 7);
   const int cv = (lane >> 3) & 1;
+  Segment pend{};  // the CTA's first segment when its stream is shared
+  int pend_h0 = 0;
+  bool has_pend = false;
   int it = 0;
   for (int k = 0; has[k & 1]; ++k) {
     if (threadIdx.x == 0) {  // one segment ahead, into the other slot
@@ -365,7 +371,32 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     consumer_sync<kCon>();
     if (!*ok_s) return;
-    finish_segment<D, G, 2>(p, sg, m_s, h0, Y, total, n, last_s, lse_f, empty_bar(held));
+    write_segment<D, G, 2>(p, sg, m_s, h0);
+    // A shared stream is counted (and merged by its last CTA) only once this CTA's range is
+    // done, so that the consumers go straight on to the next segment.  Slot 0 is always the
+    // CTA's first segment, slot 1 its last.
+    if (sg.slot == 0) {
+      pend = sg;
+      pend_h0 = h0;
+      has_pend = true;
+    }
+    if (has[(k + 1) & 1]) {
+      // Release the held stage; the proxy fence orders the generic writes to it before the
+      // copies that will refill it.
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      consumer_sync<kCon>();
+      if (lane == 0) mbar_arrive(empty_bar(held));
+    } else if (has_pend || sg.slot == 1) {
+      // The CTA's range is done: count its (at most two) shared streams, from two warps at
+      // once, and merge those it counted last.
+      const bool c0 = has_pend, c1 = sg.slot == 1;
+      consumer_sync<kCon>();
+      if (lane == 0 && warp < 2 && (warp == 0 ? c0 : c1)) last_s[warp] = count_partial(p, warp == 0 ? pend : sg, Y);
+      consumer_sync<kCon>();
+      const bool l0 = c0 && last_s[0], l1 = c1 && last_s[1];
+      if (l0) merge_stream<D, G>(p, pend, pend_h0, total, n);
+      if (l1) merge_stream<D, G>(p, sg, h0, total, n);
+    }
   }
 }
 
