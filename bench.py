@@ -507,7 +507,7 @@ def run_ours(args, rank, world, local):
         return {"workload": spec_name, "ms": ms, "GB/s": gbs, "kv_bytes": g["kv_bytes"], "bytes": g["bytes"],
                 "frac": gbs / hbm, "peak_gbs": hbm, "peak_source": peak_src, "bound": "hbm",
                 "traffic": profile_traffic(prof),
-                "kernels": ["decode_kernel (balanced split partials + merge by the last CTA of a stream)"]}
+                "kernels": ["decode_mma_kernel (tensor-core consumers, balanced split partials merged by the last CTA of a stream)"]}
 
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
