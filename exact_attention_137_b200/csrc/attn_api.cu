@@ -66,15 +66,17 @@ bool make_tmap_bf16(CUtensorMap* map, const void* base, int D, int rows, long lo
 }
 
 // A KV cache [Z, R, D] bf16 (Z = blocks * Hkv, R = rows of a block) viewed as 3-D (D, R, Z);
-// 64-column x 16-row boxes with the 128-byte swizzle.  Rows past R read as zero.
-bool make_tmap_cache(CUtensorMap* map, const void* base, int D, int R, long long Z) {
+// boxes of 128 bytes x 16 rows with the 128-byte swizzle.  Rows past R read as zero.  elem_bytes:
+// 2 (bf16) or 1 (E4M3 codes).
+bool make_tmap_cache(CUtensorMap* map, const void* base, int D, int R, long long Z, int elem_bytes = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)R, (cuuint64_t)Z};
-  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)R * D * 2};
-  cuuint32_t box[3] = {64, (cuuint32_t)attn::dec::kGranule, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)D * elem_bytes, (cuuint64_t)R * D * elem_bytes};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / elem_bytes), (cuuint32_t)attn::dec::kGranule, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box,
                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
@@ -269,13 +271,13 @@ int dispatch_decode_g(const attn::dec::Params& p, int G, int ctas, cudaStream_t 
   }
 }
 
-template <int D, int G>
+template <int D, int G, int KVB>
 int launch_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const attn::dec::Params& p, int ctas,
                       cudaStream_t st) {
-  using Lay = attn::dec::MmaLayout<D, G>;
-  auto kern = attn::dec::decode_mma_kernel<D, G>;
-  const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3);
-  static bool done[64][8] = {};
+  using Lay = attn::dec::MmaLayout<D, G, KVB>;
+  auto kern = attn::dec::decode_mma_kernel<D, G, KVB>;
+  const int key = (D == 64 ? 0 : 4) + (G == 1 ? 0 : G == 2 ? 1 : G == 4 ? 2 : 3) + (KVB == 1 ? 8 : 0);
+  static bool done[64][16] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -295,10 +297,21 @@ template <int D>
 int dispatch_decode_mma(const CUtensorMap& tk, const CUtensorMap& tv, const attn::dec::Params& p, int G, int ctas,
                         cudaStream_t st) {
   switch (G) {
-    case 1: return launch_decode_mma<D, 1>(tk, tv, p, ctas, st);
-    case 2: return launch_decode_mma<D, 2>(tk, tv, p, ctas, st);
-    case 4: return launch_decode_mma<D, 4>(tk, tv, p, ctas, st);
-    case 8: return launch_decode_mma<D, 8>(tk, tv, p, ctas, st);
+    case 1: return launch_decode_mma<D, 1, 2>(tk, tv, p, ctas, st);
+    case 2: return launch_decode_mma<D, 2, 2>(tk, tv, p, ctas, st);
+    case 4: return launch_decode_mma<D, 4, 2>(tk, tv, p, ctas, st);
+    case 8: return launch_decode_mma<D, 8, 2>(tk, tv, p, ctas, st);
+    default: return ATTN_ERR_UNSUPPORTED;
+  }
+}
+
+// E4M3 caches on the tensor-core consumers: D = 128 and at most 4 query heads per CTA.
+int dispatch_decode_mma_fp8(const CUtensorMap& tk, const CUtensorMap& tv, const attn::dec::Params& p, int G,
+                            int ctas, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_decode_mma<128, 1, 1>(tk, tv, p, ctas, st);
+    case 2: return launch_decode_mma<128, 2, 1>(tk, tv, p, ctas, st);
+    case 4: return launch_decode_mma<128, 4, 1>(tk, tv, p, ctas, st);
     default: return ATTN_ERR_UNSUPPORTED;
   }
 }
@@ -581,17 +594,24 @@ int decode_impl(const void* q, const void* k_cache, const void* v_cache, const i
   p.lse = lse;
   cudaStream_t st = as_stream(stream);
   const int ctas = plan_ctas(pl, sms);
-  if (kv_fp8) return dispatch_decode_fp8(p, pl.G, ctas, st);
-  // bf16 caches whose 16-token runs are contiguous rows (a dense cache, or pages of a
-  // multiple of 16 tokens) take the tensor-core consumers; other page sizes the fp32 ones.
+  // Caches whose 16-token runs are contiguous rows (a dense cache, or pages of a multiple of
+  // 16 tokens) take the tensor-core consumers; other page sizes the fp32 ones.
   const long long z = (long long)num_blocks * Hkv;
-  if (block_size % attn::dec::kGranule == 0 || !block_table) {
+  if ((block_size % attn::dec::kGranule == 0 || !block_table) && z < (1LL << 31)) {
     CUtensorMap tk, tv;
-    if (z < (1LL << 31) && make_tmap_cache(&tk, k_cache, D, block_size, z) &&
-        make_tmap_cache(&tv, v_cache, D, block_size, z))
+    const int eb = kv_fp8 ? 1 : 2;
+    if (make_tmap_cache(&tk, k_cache, D, block_size, z, eb) && make_tmap_cache(&tv, v_cache, D, block_size, z, eb)) {
+      if (kv_fp8) {
+        // E4M3 codes widen exactly to f16 on the tensor-core path: only the scales fold in.
+        p.scale_log2 = scale * attn::kLog2e * k_scale;
+        p.v_fac = v_scale;
+        return dispatch_decode_mma_fp8(tk, tv, p, pl.G, ctas, st);
+      }
       return D == 64 ? dispatch_decode_mma<64>(tk, tv, p, pl.G, ctas, st)
                      : dispatch_decode_mma<128>(tk, tv, p, pl.G, ctas, st);
+    }
   }
+  if (kv_fp8) return dispatch_decode_fp8(p, pl.G, ctas, st);
   return D == 64 ? dispatch_decode_g<64>(p, pl.G, ctas, st) : dispatch_decode_g<128>(p, pl.G, ctas, st);
 }
 

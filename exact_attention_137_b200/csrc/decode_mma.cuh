@@ -34,9 +34,11 @@ namespace dec {
 constexpr int kGranule = 16;  // tokens per consumer warp and stage
 static_assert(kGranule * kConsumerWarps == kStageTokens, "one granule per consumer warp");
 
-template <int D, int G>
+template <int D, int G, int KVB>
 struct MmaLayout {
-  static constexpr int kHalves = D / 64;                     // 128-byte swizzled column halves of a row
+  // E4M3 stages are half the bytes, so an E4M3 ring holds twice as many in the same memory.
+  static constexpr int kNS = KVB == 1 ? 2 * kStages : kStages;
+  static constexpr int kHalves = D * KVB / 128;              // 128-byte swizzled column blocks of a row
   static constexpr int kHalfBytes = kStageTokens * 128;      // one half of a stage's K (or V)
   static constexpr int kGranHalfBytes = kGranule * 128;      // one half of one granule
   static constexpr int kStageBytes = kHalves * kHalfBytes;   // K (or V) of one stage
@@ -44,9 +46,9 @@ struct MmaLayout {
   static constexpr int kGranTx = 2 * kHalves * kGranHalfBytes;  // bytes a granule's loads deliver
   static constexpr int kQRow = D * 2;
   static constexpr int kQBytes = G * kQRow;
-  static constexpr int kQ = kStages * kSlotBytes;
-  static constexpr int kBar = kQ + kStages * kQBytes;
-  static constexpr int kMisc = kBar + 2 * kStages * 8;
+  static constexpr int kQ = kNS * kSlotBytes;
+  static constexpr int kBar = kQ + kNS * kQBytes;
+  static constexpr int kMisc = kBar + 2 * kNS * 8;
   static constexpr int kSeg = kMisc + 64;
   static constexpr int kBytes = kSeg + 128;
   static constexpr int kAlloc = kBytes + 1024;  // the base is aligned up to 1024 bytes (swizzle atom)
@@ -55,9 +57,8 @@ struct MmaLayout {
   static_assert(sizeof(SegSlots) <= kBytes - kSeg, "segment slots fit");
 };
 
-// Byte offset of 16-byte chunk c (0 .. D/8-1) of row r in a stage's K or V: the row's two
-// 64-column halves live in separate 128-byte-swizzled blocks of 64 rows.
-template <int D>
+// Byte offset of 16-byte chunk c of row r in a stage's K or V: each 128 bytes of a row (64
+// bf16 or 128 E4M3 columns) live in a separate 128-byte-swizzled block of 64 rows.
 __device__ __forceinline__ uint32_t sw_off(int r, int c) {
   return (uint32_t)((c >> 3) * (kStageTokens * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
@@ -68,13 +69,15 @@ __device__ __forceinline__ float shfl_max_rows(float v) {
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
 }
 
-template <int D, int G>
+template <int D, int G, int KVB>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const Params p) {
   static_assert(G >= 1 && G <= 8, "the heads are the N = 8 side of the MMA");
   static_assert(D == 64 || D == 128, "head dim");
-  using L = MmaLayout<D, G>;
+  static_assert(KVB == 2 || D == 128, "E4M3 caches: D = 128");
+  using L = MmaLayout<D, G, KVB>;
+  constexpr int NS = L::kNS;
   constexpr int KS = D / 16;  // k-steps of S^T and m-tiles of O^T
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -82,7 +85,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (sbase - raw);
   auto full_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * s; };
-  auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (kStages + s); };
+  auto empty_bar = [&](int s) -> uint32_t { return sbase + L::kBar + 8u * (NS + s); };
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc);
   volatile int* ok_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
   volatile int* last_s = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), kConsumerWarps);
     }
@@ -135,8 +138,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     const int bs = p.block_size;
     const bool paged = p.block_table != nullptr;
-    int last_fill[kStages];
-    for (int s = 0; s < kStages; ++s) last_fill[s] = -1;
+    int last_fill[NS];
+    for (int s = 0; s < NS; ++s) last_fill[s] = -1;
     int it = 0;
     bool alive = true;
     Segment sg;
@@ -156,8 +159,8 @@ __global__ void __launch_bounds__(kThreads, 2)
       int cur_id = load_id(cur_first + lane);
       int nxt_id = load_id(nxt_first + lane);
       for (int st = 0; st < nst; ++st, ++it) {
-        const int s = it % kStages;
-        const int f = it / kStages;
+        const int s = it % NS;
+        const int f = it / NS;
         if (f > 0) {
           alive = __all_sync(0xffffffffu, mbar_wait(empty_bar(s), (f - 1) & 1, abort_flag));
           if (!alive) break;
@@ -190,8 +193,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
               for (int hf = 0; hf < L::kHalves; ++hf) {
                 const uint32_t off = hf * L::kHalfBytes + q * L::kGranHalfBytes;
-                tma_load_3d(dk + off, &tmK, full_bar(s), 64 * hf, slot, z);
-                tma_load_3d(dv + off, &tmV, full_bar(s), 64 * hf, slot, z);
+                tma_load_3d(dk + off, &tmK, full_bar(s), hf * (128 / KVB), slot, z);
+                tma_load_3d(dv + off, &tmV, full_bar(s), hf * (128 / KVB), slot, z);
               }
             }
           }
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (*abort_flag && lane == 0) {
       // Consumers gave up: let copies already in flight land before the CTA exits.
       int never = 0;
-      for (int s = 0; s < kStages; ++s)
+      for (int s = 0; s < NS; ++s)
         if (last_fill[s] >= 0) mbar_wait(full_bar(s), last_fill[s] & 1, &never, 100000000ull);
     }
     return;
@@ -249,21 +252,51 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int mt = 0; mt < KS; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // heads 2 t4 and 2 t4 + 1
+    float cs = c;  // score scale (times 2^-qs for E4M3 caches)
 
     bool ok = true;
     int held = 0;
     for (int st = 0; st < nst; ++st) {
-      const int s = it % kStages;
-      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / kStages) & 1, abort_flag));
+      const int s = it % NS;
+      ok = __all_sync(0xffffffffu, mbar_wait(full_bar(s), (it / NS) & 1, abort_flag));
       if (!ok) break;
       ++it;
       held = s;
       if (st == 0) {
         const uint8_t* sq = smem + L::kQ + s * L::kQBytes + g8 * L::kQRow;
+        if constexpr (KVB == 2) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          qf[ks][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 2 * t4) * 2) : 0u;
-          qf[ks][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 8 + 2 * t4) * 2) : 0u;
+          for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 2 * t4) * 2) : 0u;
+            qf[ks][1] = g8 < G ? *reinterpret_cast<const uint32_t*>(sq + (16 * ks + 8 + 2 * t4) * 2) : 0u;
+          }
+        } else {
+          // E4M3 keys enter the MMA as f16, so Q does too, scaled by 2^qs to put its largest
+          // element in [2^14, 2^15) (the scores are scaled back through cs).  k-step ks covers
+          // dims 16 ks .. 16 ks + 15; lane t4 holds dims 16 ks + 4 t4 + {0, 1} (b0) and
+          // + {2, 3} (b1), the order in which its K fragments arrive (see below).
+          float qv[KS][4];
+          float amax = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            const uint2 w = g8 < G ? *reinterpret_cast<const uint2*>(sq + (16 * ks + 4 * t4) * 2) : make_uint2(0u, 0u);
+            qv[ks][0] = bf16lo(w.x);
+            qv[ks][1] = bf16hi(w.x);
+            qv[ks][2] = bf16lo(w.y);
+            qv[ks][3] = bf16hi(w.y);
+            amax = fmaxf(amax, fmaxf(fmaxf(fabsf(qv[ks][0]), fabsf(qv[ks][1])), fmaxf(fabsf(qv[ks][2]), fabsf(qv[ks][3]))));
+          }
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+          int qs = amax > 0.f ? 14 - (((__float_as_int(amax) >> 23) & 0xFF) - 127) : 0;
+          qs = qs < -100 ? -100 : (qs > 100 ? 100 : qs);
+          const float up = __int_as_float((127 + qs) << 23), down = __int_as_float((127 - qs) << 23);
+          cs = c * down;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = pack_f16x2(qv[ks][0] * up, qv[ks][1] * up);
+            qf[ks][1] = pack_f16x2(qv[ks][2] * up, qv[ks][3] * up);
+          }
         }
       }
       const int a = a0 + st * kStageTokens + warp * kGranule;  // this warp's granule
@@ -272,17 +305,37 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t sv = sk + L::kStageBytes;
         // S^T = K Q^T, the k-steps alternating between two accumulators.
         float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (KVB == 2) {
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t af[4];
-          ldsm_x4(sk + sw_off<D>(rk, 2 * ks + ck), af[0], af[1], af[2], af[3]);
-          if (ks & 1) mma16816(so, af, qf[ks][0], qf[ks][1]);
-          else mma16816(se, af, qf[ks][0], qf[ks][1]);
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t af[4];
+            ldsm_x4(sk + sw_off(rk, 2 * ks + ck), af[0], af[1], af[2], af[3]);
+            if (ks & 1) mma16816(so, af, qf[ks][0], qf[ks][1]);
+            else mma16816(se, af, qf[ks][0], qf[ks][1]);
+          }
+        } else {
+          // One ldmatrix covers two 16-byte chunks (k-steps 2 kp, 2 kp + 1) of 16 tokens: lane
+          // (g8, t4) gets the 4 codes at dims 4 t4 .. 4 t4 + 3 of each chunk for tokens g8 and
+          // g8 + 8; the low pair is the k-step's a0 / a1, the high pair its a2 / a3.
+#pragma unroll
+          for (int kp = 0; kp < KS / 2; ++kp) {
+            uint32_t w[4];
+            ldsm_x4(sk + sw_off(rk, 2 * kp + ck), w[0], w[1], w[2], w[3]);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens g8, g8 + 8
+              const uint32_t af[4] = {e4m3x2_to_f16x2(lo_w), e4m3x2_to_f16x2(hi_w), e4m3x2_to_f16x2(lo_w >> 16),
+                                      e4m3x2_to_f16x2(hi_w >> 16)};
+              const int ks = 2 * kp + h2;
+              if (h2) mma16816_f16(so, af, qf[ks][0], qf[ks][1]);
+              else mma16816_f16(se, af, qf[ks][0], qf[ks][1]);
+            }
+          }
         }
         // x[0], x[1]: token g8, heads 2 t4, 2 t4 + 1; x[2], x[3]: token g8 + 8.
         float x[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = (se[e] + so[e]) * c;
+        for (int e = 0; e < 4; ++e) x[e] = (se[e] + so[e]) * cs;
         const bool edge = a < lo || a + kGranule > hi;  // warp-uniform
         uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;    // V fragment masks (tokens 2 t4 .., 2 t4 + 8 ..)
         if (edge) {
@@ -314,17 +367,42 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
         // P^T's B fragment: lane (g8, t4) needs P[tokens 2 t4, 2 t4 + 1 (+8)][head g8].
-        const uint32_t b0 = movmatrix_t(pack_bf16x2(p0, p1));
-        const uint32_t b1 = movmatrix_t(pack_bf16x2(p2, p3));
+        if constexpr (KVB == 2) {
+          const uint32_t b0 = movmatrix_t(pack_bf16x2(p0, p1));
+          const uint32_t b1 = movmatrix_t(pack_bf16x2(p2, p3));
 #pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          uint32_t af[4];
-          ldsm_x4_t(sv + sw_off<D>(rv, 2 * mt + cv), af[0], af[1], af[2], af[3]);
-          af[0] &= mlo;
-          af[1] &= mlo;
-          af[2] &= mhi;
-          af[3] &= mhi;
-          mma16816(acc[mt], af, b0, b1);
+          for (int mt = 0; mt < KS; ++mt) {
+            uint32_t af[4];
+            ldsm_x4_t(sv + sw_off(rv, 2 * mt + cv), af[0], af[1], af[2], af[3]);
+            af[0] &= mlo;
+            af[1] &= mlo;
+            af[2] &= mhi;
+            af[3] &= mhi;
+            mma16816(acc[mt], af, b0, b1);
+          }
+        } else {
+          const uint32_t b0 = movmatrix_t(pack_f16x2(p0, p1));
+          const uint32_t b1 = movmatrix_t(pack_f16x2(p2, p3));
+          // A transposed 8x8 read of 16-bit pairs gives lane (g8, t4) the codes of dims 2 g8 and
+          // 2 g8 + 1 for tokens 2 t4 and 2 t4 + 1 (bytes 0, 1 and 2, 3): regrouped per dim, they
+          // are the A fragments of m-tile mt (chunk mt) with row g8 = dim 2 g8 and row g8 + 8 =
+          // dim 2 g8 + 1.  One ldmatrix covers chunks 2 mp and 2 mp + 1.
+#pragma unroll
+          for (int mp = 0; mp < KS / 2; ++mp) {
+            uint32_t w[4];
+            ldsm_x4_t(sv + sw_off(rk, 2 * mp + ck), w[0], w[1], w[2], w[3]);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens 0..7, 8..15
+              uint32_t af[4] = {e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0020)), e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0031)),
+                                e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0020)), e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0031))};
+              af[0] &= mlo;
+              af[1] &= mlo;
+              af[2] &= mhi;
+              af[3] &= mhi;
+              mma16816_f16(acc[2 * mp + h2], af, b0, b1);
+            }
+          }
         }
       }
       if (st + 1 < nst) {  // the segment's last stage stays held for the merge below
@@ -358,20 +436,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
 #pragma unroll
       for (int mt = 0; mt < KS; ++mt) {
-        const int d = 16 * mt + g8;
+        // Rows g8 and g8 + 8 of m-tile mt: dims 16 mt + g8 and + 8 (bf16), or 16 mt + 2 g8 and
+        // + 1 (E4M3, the order its V fragments were built in).
+        const int d = KVB == 2 ? 16 * mt + g8 : 16 * mt + 2 * g8;
+        const int d2 = KVB == 2 ? d + 8 : d + 1;
         if (hA < G) {
           a_s[(warp * G + hA) * D + d] = acc[mt][0];
-          a_s[(warp * G + hA) * D + d + 8] = acc[mt][2];
+          a_s[(warp * G + hA) * D + d2] = acc[mt][2];
         }
         if (hB < G) {
           a_s[(warp * G + hB) * D + d] = acc[mt][1];
-          a_s[(warp * G + hB) * D + d + 8] = acc[mt][3];
+          a_s[(warp * G + hB) * D + d2] = acc[mt][3];
         }
       }
     }
     consumer_sync<kCon>();
     if (!*ok_s) return;
-    write_segment<D, G, 2>(p, sg, m_s, h0);
+    write_segment<D, G, KVB>(p, sg, m_s, h0);
     // A shared stream is counted (and merged by its last CTA) only once this CTA's range is
     // done, so that the consumers go straight on to the next segment.  Slot 0 is always the
     // CTA's first segment, slot 1 its last.
