@@ -36,10 +36,13 @@ static_assert(kGranule * kConsumerWarps == kStageTokens, "one granule per consum
 
 template <int D, int G, int KVB>
 struct MmaLayout {
-  // E4M3 stages are half the bytes, so an E4M3 ring holds twice as many in the same memory.
-  static constexpr int kNS = KVB == 1 ? 2 * kStages : kStages;
+  // E4M3 rows are half the bytes, so an E4M3 stage holds twice the tokens in the same memory
+  // (each consumer warp then takes two granules per stage).
+  static constexpr int kNS = kStages;
+  static constexpr int kTPS = KVB == 1 ? 2 * kStageTokens : kStageTokens;  // tokens per stage
+  static constexpr int kGran = kTPS / kGranule;                           // granules per stage
   static constexpr int kHalves = D * KVB / 128;              // 128-byte swizzled column blocks of a row
-  static constexpr int kHalfBytes = kStageTokens * 128;      // one half of a stage's K (or V)
+  static constexpr int kHalfBytes = kTPS * 128;              // one such block of a stage's K (or V)
   static constexpr int kGranHalfBytes = kGranule * 128;      // one half of one granule
   static constexpr int kStageBytes = kHalves * kHalfBytes;   // K (or V) of one stage
   static constexpr int kSlotBytes = 2 * kStageBytes;         // K, then V
@@ -78,6 +81,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   static_assert(KVB == 2 || D == 128, "E4M3 caches: D = 128");
   using L = MmaLayout<D, G, KVB>;
   constexpr int NS = L::kNS;
+  constexpr int TPS = L::kTPS;
+  constexpr int GPW = L::kGran / kConsumerWarps;  // granules per consumer warp and stage
   constexpr int KS = D / 16;  // k-steps of S^T and m-tiles of O^T
 
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -153,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int base = seg_base(sg);
       const int lo = base + sg.tok0, hi = base + sg.tok1;
       const int a0 = lo & ~(kGranule - 1);
-      const int nst = (hi - a0 + kStageTokens - 1) / kStageTokens;
+      const int nst = (hi - a0 + TPS - 1) / TPS;
       int cur_first = a0 / bs;
       int nxt_first = cur_first + 32;
       int cur_id = load_id(cur_first + lane);
@@ -172,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           bulk_load(sbase + L::kQ + s * L::kQBytes, p.q + ((size_t)sg.b * p.Hq + h0) * D, (uint32_t)L::kQBytes,
                     full_bar(s));
         }
-        for (int q = 0; q < kConsumerWarps; ++q) {
-          const int a = a0 + st * kStageTokens + q * kGranule;  // the granule's first position
+        for (int q = 0; q < L::kGran; ++q) {
+          const int a = a0 + st * TPS + q * kGranule;  // the granule's first position
           if (a >= hi) break;
           const int page = a / bs;
           const int slot = a - page * bs;
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int base = seg_base(sg);
     const int lo = base + sg.tok0, hi = base + sg.tok1;
     const int a0 = lo & ~(kGranule - 1);
-    const int nst = (hi - a0 + kStageTokens - 1) / kStageTokens;
+    const int nst = (hi - a0 + TPS - 1) / TPS;
     uint32_t qf[KS][2];  // B fragments of Q^T (k = dims, n = heads); heads >= G are zero
     float acc[KS][4];    // O^T tiles: rows = dims 16 mt + g8 (+8), columns = heads 2 t4, 2 t4 + 1
 #pragma unroll
@@ -299,64 +304,89 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      const int a = a0 + st * kStageTokens + warp * kGranule;  // this warp's granule
-      if (a < hi) {
+      // This warp's granules of the stage, w, w + 4, ..., processed together so that their MMA
+      // chains overlap; they share one max update per head.
+      int ga[GPW];
+#pragma unroll
+      for (int u = 0; u < GPW; ++u) ga[u] = a0 + st * TPS + (warp + kConsumerWarps * u) * kGranule;
+      if (ga[0] < hi) {
         const uint32_t sk = sbase + s * L::kSlotBytes;
         const uint32_t sv = sk + L::kStageBytes;
-        // S^T = K Q^T, the k-steps alternating between two accumulators.
-        float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (KVB == 2) {
+        float x[GPW][4];                     // [u][0..1]: token g8, heads 2 t4, 2 t4 + 1; [u][2..3]: token g8 + 8
+        uint32_t mlo[GPW], mhi[GPW];          // V fragment masks (tokens 2 t4 .., 2 t4 + 8 ..)
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) {
-            uint32_t af[4];
-            ldsm_x4(sk + sw_off(rk, 2 * ks + ck), af[0], af[1], af[2], af[3]);
-            if (ks & 1) mma16816(so, af, qf[ks][0], qf[ks][1]);
-            else mma16816(se, af, qf[ks][0], qf[ks][1]);
-          }
-        } else {
-          // One ldmatrix covers two 16-byte chunks (k-steps 2 kp, 2 kp + 1) of 16 tokens: lane
-          // (g8, t4) gets the 4 codes at dims 4 t4 .. 4 t4 + 3 of each chunk for tokens g8 and
-          // g8 + 8; the low pair is the k-step's a0 / a1, the high pair its a2 / a3.
+        for (int u = 0; u < GPW; ++u) {
+          const int a = ga[u];
+          const int rku = rk + kConsumerWarps * kGranule * u;
+          // S^T = K Q^T, the k-steps alternating between two accumulators.
+          float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};
+          if (a < hi) {  // warp-uniform
+            if constexpr (KVB == 2) {
 #pragma unroll
-          for (int kp = 0; kp < KS / 2; ++kp) {
-            uint32_t w[4];
-            ldsm_x4(sk + sw_off(rk, 2 * kp + ck), w[0], w[1], w[2], w[3]);
+              for (int ks = 0; ks < KS; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(sk + sw_off(rku, 2 * ks + ck), af[0], af[1], af[2], af[3]);
+                if (ks & 1) mma16816(so, af, qf[ks][0], qf[ks][1]);
+                else mma16816(se, af, qf[ks][0], qf[ks][1]);
+              }
+            } else {
+              // One ldmatrix covers two 16-byte chunks (k-steps 2 kp, 2 kp + 1) of 16 tokens:
+              // lane (g8, t4) gets the 4 codes at dims 4 t4 .. 4 t4 + 3 of each chunk for tokens
+              // g8 and g8 + 8; the low pair is the k-step's a0 / a1, the high pair its a2 / a3.
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens g8, g8 + 8
-              const uint32_t af[4] = {e4m3x2_to_f16x2(lo_w), e4m3x2_to_f16x2(hi_w), e4m3x2_to_f16x2(lo_w >> 16),
-                                      e4m3x2_to_f16x2(hi_w >> 16)};
-              const int ks = 2 * kp + h2;
-              if (h2) mma16816_f16(so, af, qf[ks][0], qf[ks][1]);
-              else mma16816_f16(se, af, qf[ks][0], qf[ks][1]);
+              for (int kp = 0; kp < KS / 2; ++kp) {
+                uint32_t w[4];
+                ldsm_x4(sk + sw_off(rku, 2 * kp + ck), w[0], w[1], w[2], w[3]);
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                  const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens g8, g8 + 8
+                  const uint32_t af[4] = {e4m3x2_to_f16x2(lo_w), e4m3x2_to_f16x2(hi_w), e4m3x2_to_f16x2(lo_w >> 16),
+                                          e4m3x2_to_f16x2(hi_w >> 16)};
+                  const int ks = 2 * kp + h2;
+                  if (h2) mma16816_f16(so, af, qf[ks][0], qf[ks][1]);
+                  else mma16816_f16(se, af, qf[ks][0], qf[ks][1]);
+                }
+              }
             }
           }
-        }
-        // x[0], x[1]: token g8, heads 2 t4, 2 t4 + 1; x[2], x[3]: token g8 + 8.
-        float x[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = (se[e] + so[e]) * cs;
-        const bool edge = a < lo || a + kGranule > hi;  // warp-uniform
-        uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;    // V fragment masks (tokens 2 t4 .., 2 t4 + 8 ..)
-        if (edge) {
-          const int ta = a + g8, tb = ta + 8;
-          if (!(ta >= lo && ta < hi)) x[0] = x[1] = -INFINITY;
-          if (!(tb >= lo && tb < hi)) x[2] = x[3] = -INFINITY;
-          const int t0 = a + 2 * t4;
-          mlo = (t0 >= lo && t0 < hi ? 0x0000ffffu : 0u) | (t0 + 1 >= lo && t0 + 1 < hi ? 0xffff0000u : 0u);
-          mhi = (t0 + 8 >= lo && t0 + 8 < hi ? 0x0000ffffu : 0u) | (t0 + 9 >= lo && t0 + 9 < hi ? 0xffff0000u : 0u);
+          for (int e = 0; e < 4; ++e) x[u][e] = (se[e] + so[e]) * cs;
+          mlo[u] = mhi[u] = 0xffffffffu;
+          if (a < lo || a + kGranule > hi) {  // warp-uniform: masks at the segment's ends
+            const int ta = a + g8, tb = ta + 8;
+            if (!(ta >= lo && ta < hi)) x[u][0] = x[u][1] = -INFINITY;
+            if (!(tb >= lo && tb < hi)) x[u][2] = x[u][3] = -INFINITY;
+            const int t0 = a + 2 * t4;
+            mlo[u] = (t0 >= lo && t0 < hi ? 0x0000ffffu : 0u) | (t0 + 1 >= lo && t0 + 1 < hi ? 0xffff0000u : 0u);
+            mhi[u] = (t0 + 8 >= lo && t0 + 8 < hi ? 0x0000ffffu : 0u) | (t0 + 9 >= lo && t0 + 9 < hi ? 0xffff0000u : 0u);
+          }
         }
-        // Online softmax per head; every granule holds an attended token, so the new max is
+        // Online softmax per head; the first granule holds an attended token, so the new max is
         // finite and the first rescale factor is exp2(-inf) = 0.
-        const float n0 = fmaxf(m0, shfl_max_rows(fmaxf(x[0], x[2])));
-        const float n1 = fmaxf(m1, shfl_max_rows(fmaxf(x[1], x[3])));
+        float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+        for (int u = 1; u < GPW; ++u) {
+          mx0 = fmaxf(mx0, fmaxf(x[u][0], x[u][2]));
+          mx1 = fmaxf(mx1, fmaxf(x[u][1], x[u][3]));
+        }
+        const float n0 = fmaxf(m0, shfl_max_rows(mx0));
+        const float n1 = fmaxf(m1, shfl_max_rows(mx1));
         const float al0 = fast_exp2(m0 - n0), al1 = fast_exp2(m1 - n1);
         m0 = n0;
         m1 = n1;
-        const float p0 = fast_exp2(x[0] - n0), p1 = fast_exp2(x[1] - n1);
-        const float p2 = fast_exp2(x[2] - n0), p3 = fast_exp2(x[3] - n1);
-        l0 = fmaf(l0, al0, p0 + p2);
-        l1 = fmaf(l1, al1, p1 + p3);
+        float pr[GPW][4];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int u = 0; u < GPW; ++u) {
+          pr[u][0] = fast_exp2(x[u][0] - n0);
+          pr[u][1] = fast_exp2(x[u][1] - n1);
+          pr[u][2] = fast_exp2(x[u][2] - n0);
+          pr[u][3] = fast_exp2(x[u][3] - n1);
+          s0 += pr[u][0] + pr[u][2];
+          s1 += pr[u][1] + pr[u][3];
+        }
+        l0 = fmaf(l0, al0, s0);
+        l1 = fmaf(l1, al1, s1);
         if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
@@ -366,41 +396,49 @@ __global__ void __launch_bounds__(kThreads, 2)
             acc[mt][3] *= al1;
           }
         }
-        // P^T's B fragment: lane (g8, t4) needs P[tokens 2 t4, 2 t4 + 1 (+8)][head g8].
-        if constexpr (KVB == 2) {
-          const uint32_t b0 = movmatrix_t(pack_bf16x2(p0, p1));
-          const uint32_t b1 = movmatrix_t(pack_bf16x2(p2, p3));
 #pragma unroll
-          for (int mt = 0; mt < KS; ++mt) {
-            uint32_t af[4];
-            ldsm_x4_t(sv + sw_off(rv, 2 * mt + cv), af[0], af[1], af[2], af[3]);
-            af[0] &= mlo;
-            af[1] &= mlo;
-            af[2] &= mhi;
-            af[3] &= mhi;
-            mma16816(acc[mt], af, b0, b1);
-          }
-        } else {
-          const uint32_t b0 = movmatrix_t(pack_f16x2(p0, p1));
-          const uint32_t b1 = movmatrix_t(pack_f16x2(p2, p3));
-          // A transposed 8x8 read of 16-bit pairs gives lane (g8, t4) the codes of dims 2 g8 and
-          // 2 g8 + 1 for tokens 2 t4 and 2 t4 + 1 (bytes 0, 1 and 2, 3): regrouped per dim, they
-          // are the A fragments of m-tile mt (chunk mt) with row g8 = dim 2 g8 and row g8 + 8 =
-          // dim 2 g8 + 1.  One ldmatrix covers chunks 2 mp and 2 mp + 1.
+        for (int u = 0; u < GPW; ++u) {
+          if (ga[u] >= hi) continue;  // warp-uniform
+          const int rku = rk + kConsumerWarps * kGranule * u;
+          // P^T's B fragment: lane (g8, t4) needs P[tokens 2 t4, 2 t4 + 1 (+8)][head g8].
+          if constexpr (KVB == 2) {
+            const int rvu = rv + kConsumerWarps * kGranule * u;
+            const uint32_t b0 = movmatrix_t(pack_bf16x2(pr[u][0], pr[u][1]));
+            const uint32_t b1 = movmatrix_t(pack_bf16x2(pr[u][2], pr[u][3]));
 #pragma unroll
-          for (int mp = 0; mp < KS / 2; ++mp) {
-            uint32_t w[4];
-            ldsm_x4_t(sv + sw_off(rk, 2 * mp + ck), w[0], w[1], w[2], w[3]);
+            for (int mt = 0; mt < KS; ++mt) {
+              uint32_t af[4];
+              ldsm_x4_t(sv + sw_off(rvu, 2 * mt + cv), af[0], af[1], af[2], af[3]);
+              af[0] &= mlo[u];
+              af[1] &= mlo[u];
+              af[2] &= mhi[u];
+              af[3] &= mhi[u];
+              mma16816(acc[mt], af, b0, b1);
+            }
+          } else {
+            const uint32_t b0 = movmatrix_t(pack_f16x2(pr[u][0], pr[u][1]));
+            const uint32_t b1 = movmatrix_t(pack_f16x2(pr[u][2], pr[u][3]));
+            // A transposed 8x8 read of 16-bit pairs gives lane (g8, t4) the codes of dims 2 g8
+            // and 2 g8 + 1 for tokens 2 t4 and 2 t4 + 1 (bytes 0, 1 and 2, 3): regrouped per dim,
+            // they are the A fragments of m-tile mt (chunk mt) with row g8 = dim 2 g8 and row
+            // g8 + 8 = dim 2 g8 + 1.  One ldmatrix covers chunks 2 mp and 2 mp + 1.
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens 0..7, 8..15
-              uint32_t af[4] = {e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0020)), e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0031)),
-                                e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0020)), e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0031))};
-              af[0] &= mlo;
-              af[1] &= mlo;
-              af[2] &= mhi;
-              af[3] &= mhi;
-              mma16816_f16(acc[2 * mp + h2], af, b0, b1);
+            for (int mp = 0; mp < KS / 2; ++mp) {
+              uint32_t w[4];
+              ldsm_x4_t(sv + sw_off(rku, 2 * mp + ck), w[0], w[1], w[2], w[3]);
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const uint32_t lo_w = w[2 * h2], hi_w = w[2 * h2 + 1];  // tokens 0..7, 8..15
+                uint32_t af[4] = {e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0020)),
+                                  e4m3x2_to_f16x2(__byte_perm(lo_w, 0u, 0x0031)),
+                                  e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0020)),
+                                  e4m3x2_to_f16x2(__byte_perm(hi_w, 0u, 0x0031))};
+                af[0] &= mlo[u];
+                af[1] &= mlo[u];
+                af[2] &= mhi[u];
+                af[3] &= mhi[u];
+                mma16816_f16(acc[2 * mp + h2], af, b0, b1);
+              }
             }
           }
         }
