@@ -178,9 +178,14 @@ int attn_decode_window(const void* q, const void* k_cache, const void* v_cache,
  * (1 byte; sign, 4 exponent bits with bias 7, 3 mantissa bits, subnormals, no
  * infinities), in the layouts of attn_decode; the cached value is code * k_scale
  * (resp. v_scale), one positive fp32 scale per tensor.  q, o and lse are as in
- * attn_decode (bf16 q and o).  The NaN code S.1111.111 is read as the finite value 480
- * (it never propagates).  D must be 128 and Hq/Hkv must not be a multiple of 8
- * (ATTN_ERR_UNSUPPORTED otherwise).  Scores and sums are fp32, as in attn_decode.
+ * attn_decode (bf16 q and o).  D must be 128 and Hq/Hkv must not be a multiple of 8
+ * (ATTN_ERR_UNSUPPORTED otherwise).  A dense cache, or pages of a multiple of 16 tokens, run
+ * on the tensor cores: the codes widen exactly to f16, q is scaled by a power of two into
+ * f16's range (elements more than 2^28 below the largest of its heads lose precision), the
+ * probabilities enter the PV product as f16, and scores and sums accumulate in fp32.  Other
+ * page sizes run on fp32 cores.  The NaN code S.1111.111 is not a valid cache entry: the
+ * tensor-core path propagates it as NaN (the format's definition), the fp32 path reads it as
+ * 480.
  * Returns the codes of attn_decode_window, plus ATTN_ERR_ARG for a scale that is not a
  * positive finite number. */
 int attn_decode_fp8(const void* q, const void* k_cache, const void* v_cache,
