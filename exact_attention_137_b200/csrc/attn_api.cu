@@ -182,8 +182,8 @@ int launch_bwd(const attn::bwd::Params& p, cudaStream_t st) {
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   auto kdkdv = attn::bwd::dkdv_kernel<D>;
   auto kdq = attn::bwd::dq_kernel<D>;
-  const int smem_kv = 4 * kTileBytes + 2 * attn::bwd::kRows * (int)sizeof(float);
-  const int smem_q = 4 * kTileBytes;
+  const int smem_kv = 6 * kTileBytes + 4 * attn::bwd::kRows * (int)sizeof(float);
+  const int smem_q = 6 * kTileBytes;
   if (set_smem_once(kdkdv, smem_kv, D == 64 ? 4 : 5) != cudaSuccess) return ATTN_ERR_CUDA;
   if (set_smem_once(kdq, smem_q, D == 64 ? 6 : 7) != cudaSuccess) return ATTN_ERR_CUDA;
   dim3 gkv((unsigned)cdiv(p.Sk, attn::bwd::kRows), (unsigned)(p.B * p.Hkv));

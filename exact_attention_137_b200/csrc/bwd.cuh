@@ -52,6 +52,17 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N committed groups of this thread are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// One 4-byte element; zero-filled when !valid (the source address must still be mapped).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+}
 
 // Rows [row0, row0 + 64) of a [rows][D] bf16 matrix into a swizzled tile; rows past `rows`
 // are zero-filled (their source address stays inside the matrix).
@@ -125,7 +136,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kTileBytes = kRows * D * 2;
-  const uint32_t sQ = smem_u32(smem), sO = sQ + kTileBytes, sK = sO + kTileBytes, sV = sK + kTileBytes;
+  // Q, dO, then two buffers of (K, V): the next key tile loads while this one is used.
+  const uint32_t sQ = smem_u32(smem), sO = sQ + kTileBytes, sKV = sO + kTileBytes;
   const int qt = blockIdx.x, bh = blockIdx.y;
   const int b = bh / p.Hq, h = bh - b * p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
@@ -174,13 +186,24 @@ __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
       kt_lo = first <= 0 ? 0 : (int)(first / kRows);
     }
   }
-  for (int kt = kt_lo; kt < kt_hi; ++kt) {
+  auto load_kv = [&](int kt, int bf) {
+    const uint32_t dst = sKV + (uint32_t)bf * 2u * kTileBytes;
+    load_tile<D>(dst, kb, kt * kRows, p.Sk);
+    load_tile<D>(dst + kTileBytes, vb, kt * kRows, p.Sk);
+    cp_async_commit();
+  };
+  if (kt_lo < kt_hi) load_kv(kt_lo, 0);
+  int bf = 0;
+  for (int kt = kt_lo; kt < kt_hi; ++kt, bf ^= 1) {
     const int k0 = kt * kRows;
-    __syncthreads();  // the previous tile's K, V are no longer read
-    load_tile<D>(sK, kb, k0, p.Sk);
-    load_tile<D>(sV, vb, k0, p.Sk);
-    cp_async_wait_all();
+    if (kt + 1 < kt_hi) {
+      load_kv(kt + 1, bf ^ 1);
+      cp_async_wait_group<1>();  // this tile's group has landed; the next one may still be in flight
+    } else {
+      cp_async_wait_group<0>();
+    }
     __syncthreads();
+    const uint32_t sK = sKV + (uint32_t)bf * 2u * kTileBytes, sV = sK + kTileBytes;
     float s[8][4], dp[8][4];
 #pragma unroll
     for (int n = 0; n < 8; ++n)
@@ -226,6 +249,7 @@ __global__ void __launch_bounds__(kThreads) dq_kernel(const Params p) {
         mma16816(acc[2 * n2 + 1], a, bk[2], bk[3]);
       }
     }
+    __syncthreads();  // this buffer is no longer read: the prefetch two tiles on reuses it
   }
   // dQ = scale * dS K, rounded to bf16.
 #pragma unroll
@@ -244,9 +268,11 @@ template <int D>
 __global__ void __launch_bounds__(kThreads) dkdv_kernel(const Params p) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kTileBytes = kRows * D * 2;
-  const uint32_t sK = smem_u32(smem), sV = sK + kTileBytes, sQ = sV + kTileBytes, sO = sQ + kTileBytes;
-  float* s_lse = reinterpret_cast<float*>(smem + 4 * kTileBytes);  // [64] LSE * log2(e), -inf: no row
-  float* s_dl = s_lse + kRows;                                     // [64] Delta
+  // K, V, then two buffers of (Q, dO) and of the rows' LSE and Delta: the next query tile loads
+  // while this one is used.
+  const uint32_t sK = smem_u32(smem), sV = sK + kTileBytes, sQO = sV + kTileBytes;
+  float* s_lse = reinterpret_cast<float*>(smem + 6 * kTileBytes);  // [2][64] LSE (natural log)
+  float* s_dl = s_lse + 2 * kRows;                                 // [2][64] Delta
   const int kt = blockIdx.x, bkv = blockIdx.y;
   const int b = bkv / p.Hkv, kvh = bkv - b * p.Hkv;
   const int grp = p.Hq / p.Hkv;
@@ -255,7 +281,7 @@ __global__ void __launch_bounds__(kThreads) dkdv_kernel(const Params p) {
   const int k0 = kt * kRows;
   const int r0 = warp * 16;  // this warp's keys: k0 + r0 + g (+ 8)
   const size_t kvoff = ((size_t)b * p.Hkv + kvh) * p.Sk * D;
-  load_tile<D>(sK, p.k + kvoff, k0, p.Sk);
+  load_tile<D>(sK, p.k + kvoff, k0, p.Sk);  // committed with the first query tile below
   load_tile<D>(sV, p.v + kvoff, k0, p.Sk);
 
   // Query tiles whose rows see some key of this tile.
@@ -275,21 +301,42 @@ __global__ void __launch_bounds__(kThreads) dkdv_kernel(const Params p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) acck[n][e] = accv[n][e] = 0.f;
 
-  for (int hh = 0; hh < grp; ++hh) {
+  // Work list: the group's query heads times the query tiles, flattened.
+  const int nqt = qt_hi > qt_lo ? qt_hi - qt_lo : 0;
+  const int n_it = grp * nqt;
+  auto issue = [&](int it2, int bf2) {
+    const int hh = it2 / nqt, qt = qt_lo + (it2 - hh * nqt);
     const int bh = b * p.Hq + kvh * grp + hh;
-    for (int qt = qt_lo; qt < qt_hi; ++qt) {
+    const int q0 = qt * kRows;
+    const uint32_t dst = sQO + (uint32_t)bf2 * 2u * kTileBytes;
+    load_tile<D>(dst, p.q + (size_t)bh * p.Sq * D, q0, p.Sq);
+    load_tile<D>(dst + kTileBytes, p.dout + (size_t)bh * p.Sq * D, q0, p.Sq);
+    if (threadIdx.x < kRows) {
+      // Rows past Sq read as 0; visible() gives them P = 0.
+      const int i = q0 + threadIdx.x;
+      const bool in = i < p.Sq;
+      const size_t at = (size_t)bh * p.Sq + (in ? i : 0);
+      cp_async4(smem_u32(s_lse + bf2 * kRows + threadIdx.x), p.lse + at, in);
+      cp_async4(smem_u32(s_dl + bf2 * kRows + threadIdx.x), p.delta + at, in);
+    }
+    cp_async_commit();
+  };
+  if (n_it > 0) issue(0, 0);
+  int bf = 0;
+  for (int it2 = 0; it2 < n_it; ++it2, bf ^= 1) {
+    {
+      const int hh = it2 / nqt, qt = qt_lo + (it2 - hh * nqt);
       const int q0 = qt * kRows;
-      __syncthreads();  // the previous query tile is no longer read
-      load_tile<D>(sQ, p.q + (size_t)bh * p.Sq * D, q0, p.Sq);
-      load_tile<D>(sO, p.dout + (size_t)bh * p.Sq * D, q0, p.Sq);
-      if (threadIdx.x < kRows) {
-        const int i = q0 + threadIdx.x;
-        const bool in = i < p.Sq;
-        s_lse[threadIdx.x] = in ? p.lse[(size_t)bh * p.Sq + i] * kLog2e : -INFINITY;
-        s_dl[threadIdx.x] = in ? p.delta[(size_t)bh * p.Sq + i] : 0.f;
+      if (it2 + 1 < n_it) {
+        issue(it2 + 1, bf ^ 1);
+        cp_async_wait_group<1>();  // this tile's group (and K, V) has landed
+      } else {
+        cp_async_wait_group<0>();
       }
-      cp_async_wait_all();
       __syncthreads();
+      const uint32_t sQ = sQO + (uint32_t)bf * 2u * kTileBytes, sO = sQ + kTileBytes;
+      const float* lse_b = s_lse + bf * kRows;
+      const float* dl_b = s_dl + bf * kRows;
       // S^T (keys x queries) and dP^T = V dO^T for this warp's 16 keys.
       float st[8][4], dpt[8][4];
 #pragma unroll
@@ -321,11 +368,11 @@ __global__ void __launch_bounds__(kThreads) dkdv_kernel(const Params p) {
         for (int e = 0; e < 4; ++e) {
           const int j = k0 + r0 + g + 8 * (e >> 1);
           const int qc = n * 8 + 2 * t4 + (e & 1);
-          const float l2 = s_lse[qc];
+          const float l2 = lse_b[qc] * kLog2e;  // -inf: a row with no visible key
           float pr = 0.f;
           if (l2 != -INFINITY && visible(p, q0 + qc, j)) pr = fast_exp2(st[n][e] * p.scale_log2 - l2);
           pv[e] = pr;
-          dv4[e] = pr * (dpt[n][e] - s_dl[qc]);
+          dv4[e] = pr * (dpt[n][e] - dl_b[qc]);
         }
         pa[n >> 1][(n & 1) * 2 + 0] = pack_rn(pv[0], pv[1]);
         pa[n >> 1][(n & 1) * 2 + 1] = pack_rn(pv[2], pv[3]);
@@ -346,6 +393,7 @@ __global__ void __launch_bounds__(kThreads) dkdv_kernel(const Params p) {
           mma16816(acck[2 * n2 + 1], dsa[kk], bq[2], bq[3]);
         }
     }
+    __syncthreads();  // this buffer is no longer read: the prefetch two tiles on reuses it
   }
   cp_async_wait_all();  // nothing may be in flight when the CTA exits (empty query ranges)
 #pragma unroll
