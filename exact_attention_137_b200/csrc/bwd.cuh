@@ -11,7 +11,8 @@
 // 64-row query tile (looping over the key tiles it sees).  The products are warp-level
 // bf16 tensor-core MMAs (mma.sync m16n8k16, fp32 accumulation): each warp owns 16 rows of
 // the CTA's 64-row tile, P and dS are rounded to bf16 as MMA operands, everything else
-// stays fp32 until dQ, dK, dV are rounded to bf16 at the end.
+// stays fp32 until dQ, dK, dV are rounded to bf16 at the end.  The tiles a kernel streams
+// (query tiles for dK/dV, key tiles for dQ) are double-buffered with cp.async groups.
 #pragma once
 
 #include "common.cuh"
