@@ -1,25 +1,30 @@
-// Single-token decode with the consumers on the warp-level tensor cores, for bf16 caches
-// whose rows come in runs of 16 tokens: a dense cache, or a paged pool whose page size is a
-// multiple of 16 (gocoding §5's fixed-size blocks).
+// Single-token decode with the consumers on the warp-level tensor cores, for caches whose
+// rows come in runs of 16 tokens: a dense cache, or a paged pool whose page size is a
+// multiple of 16 (gocoding §5's fixed-size blocks).  bf16 caches (KVB = 2) and E4M3 caches
+// (KVB = 1, one code per element, per-tensor scales).
 //
 // The schedule, the segments, the split-KV partials and their merge are those of
 // decode_kernel (decode.cuh): only the stage layout and the consumers differ.
 //
-//  * Stages hold 64 consecutive tokens of a segment, starting at a multiple of 16 in the
-//    sequence: four 16-token granules, each one page-aligned run of rows.  warp 4 moves each
-//    granule's K and V with 3-D TMA loads (64-column boxes, 128-byte swizzle) from the pool
-//    viewed as (D, rows of a block, block * Hkv + kv head).  Granules past the segment are
-//    not loaded; tokens of a granule outside the segment are masked.
-//  * Consumer warp w owns granule w of every stage.  With the G query heads of the segment
-//    as the N = 8 side of m16n8k16 MMAs (bf16 in, fp32 accumulate):
+//  * Stages hold consecutive positions of a segment, starting at a multiple of 16 in the
+//    sequence, as 16-token granules, each one page-aligned run of rows: 64 tokens (bf16) or
+//    128 (E4M3, the same bytes).  warp 4 moves each granule's K and V with 3-D TMA loads
+//    (128-byte boxes, 128-byte swizzle) from the pool viewed as (D, rows of a block,
+//    block * Hkv + kv head).  Granules past the segment are not loaded; tokens of a granule
+//    outside the segment are masked.
+//  * Consumer warp w owns granules w, w + 4, ... of every stage.  With the G query heads of
+//    the segment as the N = 8 side of m16n8k16 MMAs (fp32 accumulate):
 //        S^T (16 tokens x 8 heads) = K (16 x D) . Q^T (D x 8)          D/16 MMAs
 //        O^T (D x 8 heads)        += V^T (D x 16 tokens) . P^T (16 x 8)  D/16 MMAs
 //    K comes from ldmatrix, V from ldmatrix.trans (the swizzle keeps both conflict-free),
-//    and P^T's fragment is the score fragment rounded to bf16 and transposed in registers
+//    and P^T's fragment is the score fragment rounded to 16 bits and transposed in registers
 //    (movmatrix).  Each lane holds the scores of two heads for two tokens; a head's max
-//    over the granule takes three shuffles.  The online softmax per head is that of the
+//    over a granule takes three shuffles.  The online softmax per head is that of the
 //    pages (CSDN «注意力变体深挖» §6.2: running max, rescale by exp(m_old - m_new)), in
-//    the log2 domain; l sums the fp32 probabilities, P enters the MMA rounded to bf16.
+//    the log2 domain; l sums the fp32 probabilities.
+//  * bf16 caches: bf16 MMAs, P rounded to bf16.  E4M3 caches: the codes widen exactly to f16
+//    in registers (every E4M3 value is a normal f16), Q is scaled by a power of two into
+//    f16's range, and the MMAs and P are f16.
 //  * About 7 warp instructions per token and KV head, against about 50 for the fp32 FFMA
 //    consumers of decode_kernel, whose issue rate bounded them.
 #pragma once
@@ -31,8 +36,8 @@
 namespace attn {
 namespace dec {
 
-constexpr int kGranule = 16;  // tokens per consumer warp and stage
-static_assert(kGranule * kConsumerWarps == kStageTokens, "one granule per consumer warp");
+constexpr int kGranule = 16;  // tokens per MMA granule
+static_assert(kGranule * kConsumerWarps == kStageTokens, "a bf16 stage is one granule per consumer warp");
 
 template <int D, int G, int KVB>
 struct MmaLayout {
