@@ -1,0 +1,63 @@
+"""Host-side checks of the numeric facts the E4M3 tensor-core decode relies on.
+
+The decode consumers widen E4M3 codes to f16 with `cvt.rn.f16x2.e4m3x2` and multiply them by
+a query that is scaled by a power of two into f16's range.  Both steps are claimed to be exact
+(or, for the query, exact above a stated floor).  These tests check the claims with numpy's
+IEEE float16, from the format's definition (oracle.e4m3_value), without a GPU.
+"""
+
+import numpy as np
+import torch
+
+from oracle import e4m3_value
+
+F16_MIN_NORMAL = 2.0 ** -14
+F16_MAX = 65504.0
+
+
+def test_every_finite_e4m3_value_is_an_exact_normal_f16():
+    for code in range(256):
+        v = e4m3_value(code)
+        if np.isnan(v):
+            continue
+        h = np.float16(v)
+        assert float(h) == v, hex(code)
+        assert v == 0.0 or abs(v) >= F16_MIN_NORMAL, hex(code)  # subnormal codes too (2^-9 and up)
+        assert abs(v) <= F16_MAX
+
+
+def _kernel_scale_exponent(amax: float) -> int:
+    # The kernel takes the fp32 exponent field of the largest |q| (floor(log2)) and aims the
+    # largest element at [2^14, 2^15), clamped to +-100.
+    if amax <= 0.0:
+        return 0
+    e = int((np.float32(amax).view(np.int32) >> 23) & 0xFF) - 127
+    return int(np.clip(14 - e, -100, 100))
+
+
+def test_query_scaling_into_f16_range_is_exact_above_the_floor():
+    gen = torch.Generator().manual_seed(11)
+    for mag in (-30, -12, -3, 0, 4, 11, 20, 60):
+        q = (torch.randn(8, 128, generator=gen) * 2.0 ** mag).to(torch.bfloat16).to(torch.float64).numpy()
+        amax = float(np.abs(q).max())
+        qs = _kernel_scale_exponent(amax)
+        scaled = q * 2.0 ** qs
+        assert 2.0 ** 14 <= np.abs(scaled).max() < 2.0 ** 15
+        h = scaled.astype(np.float16).astype(np.float64)
+        assert np.isfinite(h).all()
+        back = h * 2.0 ** -qs
+        big = np.abs(q) >= amax * 2.0 ** -28  # normal f16 after scaling: bf16's 8 bits fit in 11
+        assert np.array_equal(back[big], q[big]), mag
+        # below the floor: f16 subnormal spacing, far under bf16's own relative precision
+        assert np.abs(back - q).max() <= amax * 2.0 ** -38
+
+
+def test_widened_products_are_exact_in_fp32():
+    # |q'| < 2^15 and |k| <= 448 < 2^9: f16 x f16 products have at most 22 significant bits, so the
+    # tensor core forms them exactly in its fp32 accumulation (only the sums round).
+    codes = [c for c in range(256) if not np.isnan(e4m3_value(c))]
+    k = np.array([e4m3_value(c) for c in codes])
+    q = np.array([np.float16(x) for x in (2.0 ** 15 - 32, 1.5, -3.25e-4, 2.0 ** -14)], dtype=np.float64)
+    prod = np.outer(q, k)
+    assert np.array_equal(prod.astype(np.float32).astype(np.float64), prod)
+    assert np.abs(prod).max() < 2.0 ** 24
